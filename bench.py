@@ -1,0 +1,444 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mixtral_fp8_decode] [--T 64]
+
+A step is one call of the whole layer (route -> permute/quantise -> both expert
+contractions -> combine) through the C ABI on one batch of T tokens; the default
+workload is the Mixtral-like FP8 decode shape (H=4096, I=14336, E=8, top_k=2) at
+T=64.  Inputs are seeded synthetic tensors resident in HBM; the expert weights
+(1.41 GB) exceed the 126 MB L2, so no L2 flush is needed between steps.  W
+untimed warm-up steps, then exactly K steps timed with CUDA events on the
+launching stream between a barrier + synchronize on both sides; the time is the
+max over ranks.  For N > 1 every rank runs an independent replica of the layer
+(the single-GPU layer has no exchange step) and `value` is the tokens of all
+ranks divided by that time.
+
+Rank 0 prints one JSON line.  Besides the contract keys it reports the roofline of
+the dominant kernel (timed live per launch with CUDA events through
+fused_moe_profile), the oracle timed on the host cores (cpu_baseline), an
+end-to-end number through fused_moe_host_io with pinned host buffers, and the SM
+clocks sampled with nvidia-smi during the timed region.
+
+--impl reference times the CPU oracle (the reference arm) on the same workload:
+each step runs the oracle's expert networks for one touched expert over the full
+token batch (a bounded slice); one cycle over the touched experts plus routing and
+combine is one full layer pass.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_26_b200 import inputs as minp  # noqa: E402
+
+METRIC = "fused-MoE tokens/s; achieved HBM GB/s (decode) / FP8 TFLOPS (prefill) vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+GEMM_SOURCES = ("mixture_experts_layer_26_b200/csrc/gemm.cu",
+                "mixture_experts_layer_26_b200/csrc/fmoe_common.cuh")
+
+
+# --------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload_tag: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if it was taken
+    on the current kernel source (profiles/*.md lines 'traffic_bytes_per_launch' and
+    'source_hash'); else None."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        if not (name.startswith(kernel) and workload_tag in name and name.endswith(".md")):
+            continue
+        text = open(os.path.join(pdir, name)).read()
+        t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        hsh = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+        if t and hsh and hsh.group(1) == gemm_source_hash():
+            return float(t.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of the GPU with the given PCI bus id."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, props):
+        # nvidia-smi prints the bus id as DDDDDDDD:BB:DD.F
+        self.bus_id = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9 or not self._match(parts[0]):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+    def _match(self, bus: str) -> bool:
+        return bus.lower()[-7:] == self.bus_id[-7:]
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return 1
+
+
+def np_inputs(inp: minp.MoEInputs):
+    fp8 = inp.shape.wdtype == "fp8"
+    wb = (lambda t: t.numpy()) if fp8 else minp.bf16_bits
+    return dict(x_bits=minp.bf16_bits(inp.x), wr_bits=minp.bf16_bits(inp.router_w),
+                w13=wb(inp.w13), w2=wb(inp.w2),
+                w13_scale=None if inp.w13_scale is None else inp.w13_scale.numpy(),
+                w2_scale=None if inp.w2_scale is None else inp.w2_scale.numpy(), fp8=fp8)
+
+
+def reduce_max(dist, v: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_second(world: int, T: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes T tokens per step."""
+    return world * T * steps / (ms_max / 1e3)
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_full_pass(inp):
+    """The oracle on the whole batch once: (seconds, touched experts)."""
+    from oracle import fused_moe_oracle as O
+    d = np_inputs(inp)
+    t0 = time.perf_counter()
+    r = O.fused_moe(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], inp.shape.top_k, fp8=d["fp8"],
+                    w13_scale=d["w13_scale"], w2_scale=d["w2_scale"])
+    return time.perf_counter() - t0, int((r["counts"] > 0).sum())
+
+
+class OracleSlices:
+    """Bounded steps of the oracle: the expert networks of one touched expert over the
+    whole token batch per step, plus routing / permutation / combine once per cycle."""
+
+    def __init__(self, inp):
+        from oracle import fused_moe_oracle as O
+        self.O, self.inp, self.d = O, inp, np_inputs(inp)
+        s = inp.shape
+        t0 = time.perf_counter()
+        d = self.d
+        ids, w, _ = O.router(d["x_bits"], d["wr_bits"], s.top_k)
+        counts, offsets, rows, inv = O.permute(ids, s.E)
+        a_perm, s1, _, _ = O.permute_quant(d["x_bits"], rows, s.top_k, d["fp8"])
+        self.prep = (ids, w, counts, offsets, rows, inv, a_perm, s1)
+        self.fixed_s = time.perf_counter() - t0
+        self.touched = [e for e in range(s.E) if counts[e] > 0]
+        self.i = 0
+
+    def step(self):
+        s, d, O = self.inp.shape, self.d, self.O
+        ids, w, counts, offsets, rows, inv, a_perm, s1 = self.prep
+        e = self.touched[self.i % len(self.touched)]
+        self.i += 1
+        offs = np.zeros_like(offsets)
+        offs[e + 1:] = offsets[e + 1] - offsets[e]
+        r0, r1 = offsets[e], offsets[e + 1]
+        O.experts(a_perm[r0:r1], offs, rows[r0:r1], w, d["w13"], d["w2"], s.H, s.I, s.E, d["fp8"],
+                  s1, d["w13_scale"], d["w2_scale"])
+
+    def combine_seconds(self):
+        s = self.inp.shape
+        y = np.zeros((s.R, s.H))
+        t0 = time.perf_counter()
+        self.O.combine(y, self.prep[5], s.T, s.top_k)
+        return time.perf_counter() - t0
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    s = minp.shape(args.workload, args.T)
+    inp = minp.make_inputs(s, seed=0)
+    sl = OracleSlices(inp)
+    warm = min(args.warmup, 2)  # the oracle has no caches to warm beyond BLAS thread start-up
+    for _ in range(warm):
+        sl.step()
+    sl.i = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sl.step()
+    dt = time.perf_counter() - t0
+    cycles = args.steps / len(sl.touched)
+    total = dt + cycles * (sl.fixed_s + sl.combine_seconds())
+    value = s.T * cycles / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp64 (oracle; e4m3 codes decoded exactly)",
+        "data": "synthetic", "config": workload_config(s, "oracle"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{args.steps} steps, each the expert networks of one of the "
+                                   f"{len(sl.touched)} touched experts over all T={s.T} tokens; "
+                                   "routing/permutation/combine added once per expert cycle; "
+                                   f"{warm} of the {args.warmup} warm-up steps executed"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def workload_config(s, variant):
+    weights = 3 * s.H * s.I * s.E * (1 if s.wdtype == "fp8" else 2)
+    return {"workload": f"{s.name}: H={s.H} I={s.I} E={s.E} top_k={s.top_k} T={s.T} "
+                        f"({s.wdtype} weights)",
+            "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.top_k, "variant": variant,
+            "l2": f"inputs larger than L2: expert weights {weights / 1e9:.2f} GB vs "
+                  f"{L2_BYTES / 2 ** 20:.0f} MB L2, no flush",
+            "parallelism": "replicas (one independent layer per GPU)"}
+
+
+def run_ours(args, rank, world, local_rank):
+    from mixture_experts_layer_26_b200 import capi
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = minp.shape(args.workload, args.T)
+    fp8 = s.wdtype == "fp8"
+    inp = minp.make_inputs(s, seed=0)
+    x = inp.x.to(dev)
+    wr = inp.router_w.to(dev)
+    w13, w2 = inp.w13.to(dev), inp.w2.to(dev)
+    s13 = inp.w13_scale.to(dev) if fp8 else None
+    s2 = inp.w2_scale.to(dev) if fp8 else None
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, args.variant)
+    ws = capi.alloc_workspace(dims, dev)
+    sc = capi.make_scales(s13, s2)
+    out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        return reduce_max(dist, v, dev)
+
+    for _ in range(args.warmup):
+        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+    torch.cuda.synchronize()
+    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+
+    # ---- timed region: exactly K steps
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev)) if rank == 0 else None
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    status = capi.fused_moe_get_device_status(ws, stream)
+    assert status == capi.FMOE_OK, capi.status_string(status)
+    ms_step = ms / args.steps
+    value = tokens_per_second(world, s.T, args.steps, ms)
+
+    # ---- per-kernel times (events after every launch), same inputs, after the timed region
+    nprof = max(5, min(args.steps, 200))
+    per = {}
+    for _ in range(nprof):
+        for name, t in capi.fused_moe_profile(dims, x, wr, w13, w2, sc, out, ws, stream):
+            per.setdefault(name, []).append(t)
+    kern_ms = {k: statistics.mean(v) for k, v in per.items()}
+    _, plan = capi.fused_moe_debug_scalars(ws, stream)
+
+    # ---- end to end through the host-buffer entry point
+    x_host = inp.x.clone().pin_memory()
+    out_host = torch.empty(s.T, s.H, dtype=torch.bfloat16).pin_memory()
+    n_e2e = max(3, min(args.steps, 500))
+    for _ in range(3):
+        capi.fused_moe_host_io(dims, x_host, wr, w13, w2, sc, out_host, ws, stream)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        capi.fused_moe_host_io(dims, x_host, wr, w13, w2, sc, out_host, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = tokens_per_second(world, s.T, n_e2e, e2e_ms)
+
+    # ---- experts the batch touched, from the GPU routing + permutation steps
+    R = s.R
+    ids_d = torch.empty(R, dtype=torch.int32, device=dev)
+    tw_d = torch.empty(R, dtype=torch.float32, device=dev)
+    counts_d = torch.empty(s.E, dtype=torch.int32, device=dev)
+    offs_d = torch.empty(s.E + 1, dtype=torch.int32, device=dev)
+    rows_d = torch.empty(R, dtype=torch.int32, device=dev)
+    inv_d = torch.empty(R, dtype=torch.int32, device=dev)
+    aperm_d = torch.empty(R, s.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+    capi.fused_moe_route(dims, x, wr, ids_d, tw_d, ws, stream)
+    capi.fused_moe_permute(dims, ids_d, x, sc, counts_d, offs_d, rows_d, inv_d, aperm_d, ws, stream)
+    touched = int((counts_d > 0).sum().item())
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # ---- roofline of the dominant kernel
+    esz = 1 if fp8 else 2
+    peaks, peak_kind = load_peaks()
+    dom = max(kern_ms, key=kern_ms.get)
+    gemm1_bytes = touched * 2 * s.H * s.I * esz          # weights of the touched experts
+    gemm2_bytes = touched * s.H * s.I * esz
+    algo = {"gemm1": gemm1_bytes, "gemm2": gemm2_bytes}
+    dom_bytes = algo.get(dom.split("_")[0])
+    variant = "swap_ab" if "swapab" in "".join(kern_ms) else "normal"
+    roof = None
+    if dom_bytes is not None:
+        ach = dom_bytes / (kern_ms[dom] / 1e3) / 1e9
+        traffic = profiled_traffic(dom, f"{args.workload}_T{s.T}")
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": dom, "kernel_us": round(1e3 * kern_ms[dom], 2),
+                "algorithmic_bytes": dom_bytes,
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"}
+    step_weight_bytes = gemm1_bytes + gemm2_bytes
+    # cpu baseline: the oracle on the whole batch, once
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        secs, _ = oracle_full_pass(inp)
+        cpu = {"value": s.T / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"one full oracle pass over the T={s.T} batch ({secs:.1f} s)"}
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
+        "data": "synthetic (seeded; N(0,1) x, N(0,1/sqrt(fan_in)) weights, per-expert e4m3 scales)",
+        "config": workload_config(s, variant),
+        "roofline": roof,
+        "step_hbm": {"weight_bytes": step_weight_bytes,
+                     "achieved_gbs": round(step_weight_bytes / (ms_step / 1e3) / 1e9, 1),
+                     "frac": round(step_weight_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "touched_experts": touched},
+        "kernels_us": {k: round(1e3 * v, 2) for k, v in kern_ms.items()},
+        "plan": plan,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": s.T * s.H * 2, "d2h_bytes_per_step": s.T * s.H * 2,
+                "api": "fused_moe_host_io (pinned host x and out)"},
+        "gpu_launches": capi.fused_moe_launches_per_call(dims) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_fp8_decode", choices=sorted(minp.WORKLOADS))
+    ap.add_argument("--T", type=int, default=64)
+    ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,226 @@
+/*
+ * fused_moe.h -- C ABI of a fused Mixture-of-Experts layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer.  A fused MoE merges token routing, data shuffling and the expert-network
+ * computations into one batched GPU operation instead of separate sequential loops
+ * (readmex.ai story "AWS details fused MoE kernel optimizations on SageMaker, up to 10%
+ * throughput gain", opening section; agentic-affairs.com, "Swap-AB targets matrix
+ * execution on Hopper").  For T tokens x[T,H], E experts and top_k = k:
+ *
+ *   route:    logits = x . router_w^T (fp32), the k largest per token, weights =
+ *             softmax over all E renormalised over the k chosen experts
+ *   permute:  rows (t, j) grouped by expert (stable), activations gathered in that
+ *             order and, for FP8, quantised to e4m3 with a per-tensor scale
+ *   experts:  per expert e, h = SiLU(A_e . W1_e^T) * (A_e . W3_e^T), y = h . W2_e^T,
+ *             fp32 accumulation; FP8 weights carry one fp32 scale per expert and
+ *             tensor ("tensor-quantized" FP8: readmex.ai opening section;
+ *             agentic-affairs.com, "Triton improves the FP8 execution path"); h is
+ *             re-quantised per tensor before the second contraction; each row is
+ *             multiplied by its routing weight
+ *   combine:  out[t] = bf16( sum over j < k of y[row of (t, j)] ), in slot order
+ *
+ * Readings where the pages are silent: router logits are summed in fp32 in a fixed
+ * order (chunks of 8 columns, chunk c on lane c mod 32, ascending, then an xor
+ * butterfly 16,8,4,2,1), so expert choice is exactly reproducible; top-k ties go to
+ * the lower expert index; activation scales are amax/448 (dynamic, the default) or a
+ * static value; rows 0..I-1 of w13 are W1 (gate) and rows I..2I-1 are W3 (up).
+ *
+ * Conventions for every call.
+ *  - Pointers named "device" are CUDA device pointers, 16-byte aligned; the caller
+ *    owns all memory.  The library never allocates or frees memory and never
+ *    synchronises the stream, except in the calls documented as synchronous.
+ *  - Layouts are row-major and contiguous.  bf16 values are passed as raw 16-bit
+ *    patterns, e4m3 values as bytes (OCP e4m3fn: bias 7, max 448, no infinities).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is enqueued
+ *    asynchronously on it; results are valid once the stream reaches that point.
+ *  - Argument checks run before any CUDA call and return synchronously:
+ *      FMOE_ERR_INVALID_ARG  null dims / pointer, T < 0, H, I < 1, E < 1 or > 256,
+ *                            top_k < 1 or > E, unknown wdtype / variant, FP8 without
+ *                            weight scales
+ *      FMOE_ERR_UNSUPPORTED  H % 256 != 0, I % 128 != 0, H > 16384, a device pointer
+ *                            not 16-byte aligned, sizes whose element counts exceed
+ *                            2^31
+ *      FMOE_ERR_WORKSPACE    ws_bytes < fused_moe_workspace_size(dims), or ws not
+ *                            256-byte aligned
+ *    T == 0 returns FMOE_OK after the dims checks and launches nothing.
+ *    FMOE_ERR_CUDA reports a failed launch (cudaGetLastError after the launch).
+ *  - Device-side problems (a bounded wait that ran out: FMOE_ERR_TIMEOUT; an expert
+ *    id outside [0, E) in topk_ids: FMOE_ERR_DEVICE_BOUNDS) are recorded in a sticky
+ *    status word inside the workspace and read with fused_moe_get_device_status.
+ *  - The steps share state through the workspace: permute stores the activation
+ *    scale it used there and experts reads it back, so use one workspace (sized for
+ *    the same dims) for the steps of one call sequence.  Calls that use the same
+ *    workspace must not overlap on the GPU.
+ */
+#ifndef FUSED_MOE_H_
+#define FUSED_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FUSED_MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FMOE_API __attribute__((visibility("default")))
+#else
+#define FMOE_API
+#endif
+
+typedef enum {
+  FMOE_OK = 0,
+  FMOE_ERR_INVALID_ARG = 1,
+  FMOE_ERR_UNSUPPORTED = 2,
+  FMOE_ERR_WORKSPACE = 3,
+  FMOE_ERR_CUDA = 4,
+  FMOE_ERR_TIMEOUT = 5,
+  FMOE_ERR_DEVICE_BOUNDS = 6
+} fmoe_status;
+
+/* Storage format of the activations entering the contractions and of the weights. */
+typedef enum {
+  FMOE_BF16 = 0,     /* bf16 weights, no quantisation; h rounded to bf16 */
+  FMOE_FP8_E4M3 = 1  /* e4m3 weights with per-expert fp32 scales; e4m3 activations */
+} fmoe_wdtype;
+
+/* Tile shape of the grouped GEMMs.  AUTO picks SWAP_AB when an expert receives at
+ * most 64 rows on average (T*k/E <= 64) and NORMAL otherwise.  SWAP_AB puts 128 weight
+ * rows in the MMA's M slot and the expert's tokens in N (decode); NORMAL puts 128
+ * tokens in M and 256 weight rows in N (prefill).  Both give the same results up to
+ * fp32 summation order. */
+typedef enum { FMOE_VARIANT_AUTO = 0, FMOE_VARIANT_SWAP_AB = 1, FMOE_VARIANT_NORMAL = 2 } fmoe_variant;
+
+typedef struct {
+  int32_t T;        /* tokens */
+  int32_t H;        /* hidden size */
+  int32_t I;        /* expert intermediate size */
+  int32_t E;        /* experts */
+  int32_t top_k;    /* experts per token */
+  int32_t wdtype;   /* fmoe_wdtype */
+  int32_t variant;  /* fmoe_variant */
+} fmoe_dims;
+
+typedef struct {
+  const float* w13_scale; /* [E] device: scale of each expert's w13 (FP8 only) */
+  const float* w2_scale;  /* [E] device: scale of each expert's w2 (FP8 only) */
+  float a1_scale;         /* > 0: static activation scale; <= 0: amax(|x|)/448 */
+  float a2_scale;         /* > 0: static scale of h; <= 0: amax(|h|)/448 */
+} fmoe_scales;
+
+typedef void* fmoe_stream; /* a cudaStream_t */
+
+/* ABI version of the loaded library (FUSED_MOE_ABI_VERSION). */
+FMOE_API int32_t fused_moe_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+FMOE_API const char* fused_moe_status_string(fmoe_status status);
+
+/* Bytes of device workspace the calls below need for these dims; 0 if the dims are
+ * invalid.  Host-only, makes no CUDA call. */
+FMOE_API size_t fused_moe_workspace_size(const fmoe_dims* dims);
+
+/* Zero the workspace header (status word included).  Call once on a new workspace
+ * before its first use.  Asynchronous on `stream`. */
+FMOE_API fmoe_status fused_moe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream stream);
+
+/* Step 1, routing.
+ *   x         [T, H]  bf16, device
+ *   router_w  [E, H]  bf16, device
+ *   topk_ids  [T, k]  int32 out, device: chosen experts, by descending logit
+ *   topk_w    [T, k]  fp32 out, device: renormalised softmax weights
+ * Also records max |x| partials in ws for the FP8 activation scale. */
+FMOE_API fmoe_status fused_moe_route(const fmoe_dims* dims, const void* x, const void* router_w,
+                            int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                            fmoe_stream stream);
+
+/* Step 2, data shuffling.
+ *   topk_ids    [T*k]   int32, device (from route)
+ *   x           [T, H]  bf16, device
+ *   scales      may be NULL (dynamic activation scale); only a1_scale is read
+ *   counts      [E]     int32 out: rows per expert
+ *   offsets     [E+1]   int32 out: exclusive prefix sum of counts
+ *   sorted_rows [T*k]   int32 out: flattened indices t*k+j grouped by expert,
+ *                       ascending within an expert
+ *   inv_perm    [T*k]   int32 out: inverse of sorted_rows
+ *   a_perm      [T*k, H] out: x[sorted_rows[p] / k], as e4m3 bytes (FP8: multiplied by
+ *                       448/amax(|x|) in fp32, round to nearest even, saturating) or bf16
+ * Needs the ws that route wrote (the max |x| partials); stores the activation scale
+ * in ws for experts. */
+FMOE_API fmoe_status fused_moe_permute(const fmoe_dims* dims, const int32_t* topk_ids, const void* x,
+                              const fmoe_scales* scales, int32_t* counts, int32_t* offsets,
+                              int32_t* sorted_rows, int32_t* inv_perm, void* a_perm, void* ws,
+                              size_t ws_bytes, fmoe_stream stream);
+
+/* Step 3, the expert networks on the permuted rows.
+ *   a_perm      [T*k, H] e4m3 or bf16, device (from permute)
+ *   offsets     [E+1], sorted_rows [T*k]: from permute
+ *   topk_w      [T*k] fp32 routing weights in (t, j) order (from route)
+ *   w13         [E, 2I, H] e4m3 bytes or bf16: rows 0..I-1 = W1 (gate), I..2I-1 = W3 (up)
+ *   w2          [E, H, I]  e4m3 bytes or bf16
+ *   scales      FP8: w13_scale, w2_scale required; a2_scale read
+ *   y_perm      [T*k, H] fp32 out: row p = topk_w of its (t, j) times the expert MLP
+ *               output of a_perm[p]
+ * Uses the activation scale permute stored in ws. */
+FMOE_API fmoe_status fused_moe_experts(const fmoe_dims* dims, const void* a_perm, const int32_t* offsets,
+                              const int32_t* sorted_rows, const float* topk_w, const void* w13,
+                              const void* w2, const fmoe_scales* scales, float* y_perm, void* ws,
+                              size_t ws_bytes, fmoe_stream stream);
+
+/* Step 4, back to token order.
+ *   y_perm   [T*k, H] fp32, device;  inv_perm [T*k] int32, device
+ *   out      [T, H] bf16 out: out[t] = bf16(sum over j of y_perm[inv_perm[t*k+j]]),
+ *            fp32 adds in j order, round to nearest even
+ * Needs no workspace. */
+FMOE_API fmoe_status fused_moe_combine(const fmoe_dims* dims, const float* y_perm, const int32_t* inv_perm,
+                              void* out, fmoe_stream stream);
+
+/* The whole layer in one call: route, permute, experts, combine with every
+ * intermediate kept in ws.  x [T, H] bf16, router_w [E, H] bf16, w13, w2 as above,
+ * out [T, H] bf16; all device pointers.  No host synchronisation happens between
+ * the steps. */
+FMOE_API fmoe_status fused_moe(const fmoe_dims* dims, const void* x, const void* router_w, const void* w13,
+                      const void* w2, const fmoe_scales* scales, void* out, void* ws,
+                      size_t ws_bytes, fmoe_stream stream);
+
+/* fused_moe with x and out in HOST memory (pinned memory gives asynchronous copies):
+ * copies x to ws, runs the layer, copies out back and synchronises `stream` before
+ * returning.  Weights and scales stay device pointers. */
+FMOE_API fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host, const void* router_w,
+                              const void* w13, const void* w2, const fmoe_scales* scales,
+                              void* out_host, void* ws, size_t ws_bytes, fmoe_stream stream);
+
+/* Number of kernels one fused_moe call launches for these dims (FP8: 8 NORMAL, 10
+ * SWAP_AB; bf16: 7 NORMAL, 9 SWAP_AB; 0 for T == 0; -1 for invalid dims).  Host-only. */
+FMOE_API int32_t fused_moe_launches_per_call(const fmoe_dims* dims);
+
+/* Measurement: runs fused_moe once with a CUDA event recorded on `stream` before the
+ * first and after every kernel launch, waits for the stream, and writes the device
+ * time of launch i to ms_host[i] (milliseconds) and a static name of the kernel to
+ * names_host[i] (may be NULL), for at most `cap` launches; *n_host = launches
+ * written.  Synchronous.  Creates its CUDA events on first use. */
+FMOE_API fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, const void* router_w,
+                                       const void* w13, const void* w2, const fmoe_scales* scales,
+                                       void* out, void* ws, size_t ws_bytes, fmoe_stream stream,
+                                       float* ms_host, const char** names_host, int32_t cap,
+                                       int32_t* n_host);
+
+/* Synchronous: waits for `stream`, then returns the sticky device status recorded in
+ * ws (FMOE_OK, FMOE_ERR_TIMEOUT or FMOE_ERR_DEVICE_BOUNDS), or FMOE_ERR_CUDA if the
+ * wait or copy failed. */
+FMOE_API fmoe_status fused_moe_get_device_status(const void* ws, fmoe_stream stream);
+
+/* Synchronous: copies the scalars of the last call in ws to host memory:
+ *   f[0..5] = amax|x|, s1, 448/amax|x| (or 1/s1), amax|h|, s2, inverse of s2
+ *   i[0..2] = expert row chunks, split-K of the first and of the second contraction
+ * Either pointer may be NULL. */
+FMOE_API fmoe_status fused_moe_debug_scalars(const void* ws, float* f6_host, int32_t* i3_host,
+                                    fmoe_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FUSED_MOE_H_ */

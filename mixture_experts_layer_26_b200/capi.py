@@ -1,0 +1,255 @@
+"""ctypes binding of libfused_moe.so (include/fused_moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch supplies device memory (tensor.data_ptr()) and streams.  Importing
+this module fails loudly when the library has not been built; there is no fallback.
+
+Low-level functions keep the C names (fused_moe_route, fused_moe_permute,
+fused_moe_experts, fused_moe_combine, fused_moe, fused_moe_host_io, ...) and take
+torch tensors; `FusedMoE` wraps a workspace for repeated one-call use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int32, c_size_t, c_void_p
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfused_moe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_26_b200.build` "
+        "(the fused MoE layer has no CPU or Python fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_WORKSPACE = 0, 1, 2, 3
+FMOE_ERR_CUDA, FMOE_ERR_TIMEOUT, FMOE_ERR_DEVICE_BOUNDS = 4, 5, 6
+FMOE_BF16, FMOE_FP8_E4M3 = 0, 1
+VARIANTS = {"auto": 0, "swap_ab": 1, "normal": 2}
+
+EXPORTED = (
+    "fused_moe_abi_version", "fused_moe_status_string", "fused_moe_workspace_size",
+    "fused_moe_workspace_init", "fused_moe_route", "fused_moe_permute", "fused_moe_experts",
+    "fused_moe_combine", "fused_moe", "fused_moe_host_io", "fused_moe_get_device_status",
+    "fused_moe_debug_scalars", "fused_moe_launches_per_call", "fused_moe_profile",
+)
+
+
+class FmoeDims(ctypes.Structure):
+    _fields_ = [("T", c_int32), ("H", c_int32), ("I", c_int32), ("E", c_int32),
+                ("top_k", c_int32), ("wdtype", c_int32), ("variant", c_int32)]
+
+
+class FmoeScales(ctypes.Structure):
+    _fields_ = [("w13_scale", c_void_p), ("w2_scale", c_void_p),
+                ("a1_scale", c_float), ("a2_scale", c_float)]
+
+
+def _sig(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_DP = POINTER(FmoeDims)
+_SP = POINTER(FmoeScales)
+_abi = _sig("fused_moe_abi_version", c_int32)
+_status_string = _sig("fused_moe_status_string", c_char_p, c_int32)
+_ws_size = _sig("fused_moe_workspace_size", c_size_t, _DP)
+_ws_init = _sig("fused_moe_workspace_init", c_int32, c_void_p, c_size_t, c_void_p)
+_route = _sig("fused_moe_route", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+              c_size_t, c_void_p)
+_permute = _sig("fused_moe_permute", c_int32, _DP, c_void_p, c_void_p, _SP, c_void_p, c_void_p,
+                c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p)
+_experts = _sig("fused_moe_experts", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                c_void_p, _SP, c_void_p, c_void_p, c_size_t, c_void_p)
+_combine = _sig("fused_moe_combine", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p)
+_fused = _sig("fused_moe", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP, c_void_p,
+              c_void_p, c_size_t, c_void_p)
+_host_io = _sig("fused_moe_host_io", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
+                c_void_p, c_void_p, c_size_t, c_void_p)
+_dev_status = _sig("fused_moe_get_device_status", c_int32, c_void_p, c_void_p)
+_dbg = _sig("fused_moe_debug_scalars", c_int32, c_void_p, POINTER(c_float), POINTER(c_int32),
+            c_void_p)
+_launches = _sig("fused_moe_launches_per_call", c_int32, _DP)
+_profile = _sig("fused_moe_profile", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
+                c_void_p, c_void_p, c_size_t, c_void_p, POINTER(c_float), POINTER(c_char_p),
+                c_int32, POINTER(c_int32))
+
+
+class FusedMoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def abi_version() -> int:
+    return int(_abi())
+
+
+def status_string(status: int) -> str:
+    return _status_string(int(status)).decode()
+
+
+def _check(st: int, where: str) -> int:
+    if st != FMOE_OK:
+        raise FusedMoEError(st, where)
+    return st
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def make_dims(T: int, H: int, I: int, E: int, top_k: int, fp8: bool, variant: str = "auto") -> FmoeDims:
+    return FmoeDims(T, H, I, E, top_k, FMOE_FP8_E4M3 if fp8 else FMOE_BF16, VARIANTS[variant])
+
+
+def dims_of(x: torch.Tensor, w13: torch.Tensor, top_k: int, variant: str = "auto") -> FmoeDims:
+    """Dims from x [T,H] and w13 [E,2I,H] (uint8 = e4m3 bytes, bfloat16 = bf16)."""
+    T, H = x.shape
+    E, twoI, H2 = w13.shape
+    assert H2 == H and twoI % 2 == 0
+    return make_dims(T, H, twoI // 2, E, top_k, w13.dtype == torch.uint8, variant)
+
+
+def make_scales(w13_scale=None, w2_scale=None, a1_scale: float = 0.0, a2_scale: float = 0.0) -> FmoeScales:
+    return FmoeScales(_ptr(w13_scale), _ptr(w2_scale), float(a1_scale), float(a2_scale))
+
+
+def workspace_size(dims: FmoeDims) -> int:
+    return int(_ws_size(ctypes.byref(dims)))
+
+
+def alloc_workspace(dims: FmoeDims, device="cuda") -> torch.Tensor:
+    """A workspace tensor (uint8, 256-byte aligned by the caching allocator), initialised."""
+    n = workspace_size(dims)
+    if n == 0:
+        raise FusedMoEError(FMOE_ERR_INVALID_ARG, "workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(_ws_init(ws.data_ptr(), n, _stream(None)), "fused_moe_workspace_init")
+    return ws
+
+
+def fused_moe_workspace_init(ws: torch.Tensor, stream=None) -> int:
+    return _check(_ws_init(ws.data_ptr(), ws.numel(), _stream(stream)), "fused_moe_workspace_init")
+
+
+def fused_moe_route(dims, x, router_w, topk_ids, topk_w, ws, stream=None, check=True) -> int:
+    st = _route(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(topk_ids), _ptr(topk_w),
+                _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_route") if check else st
+
+
+def fused_moe_permute(dims, topk_ids, x, scales, counts, offsets, sorted_rows, inv_perm, a_perm,
+                      ws, stream=None, check=True) -> int:
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _permute(ctypes.byref(dims), _ptr(topk_ids), _ptr(x), sp, _ptr(counts), _ptr(offsets),
+                  _ptr(sorted_rows), _ptr(inv_perm), _ptr(a_perm), _ptr(ws),
+                  ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_permute") if check else st
+
+
+def fused_moe_experts(dims, a_perm, offsets, sorted_rows, topk_w, w13, w2, scales, y_perm, ws,
+                      stream=None, check=True) -> int:
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _experts(ctypes.byref(dims), _ptr(a_perm), _ptr(offsets), _ptr(sorted_rows), _ptr(topk_w),
+                  _ptr(w13), _ptr(w2), sp, _ptr(y_perm), _ptr(ws),
+                  ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_experts") if check else st
+
+
+def fused_moe_combine(dims, y_perm, inv_perm, out, stream=None, check=True) -> int:
+    st = _combine(ctypes.byref(dims), _ptr(y_perm), _ptr(inv_perm), _ptr(out), _stream(stream))
+    return _check(st, "fused_moe_combine") if check else st
+
+
+def fused_moe(dims, x, router_w, w13, w2, scales, out, ws, stream=None, check=True) -> int:
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _fused(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(w13), _ptr(w2), sp, _ptr(out),
+                _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe") if check else st
+
+
+def fused_moe_host_io(dims, x_host, router_w, w13, w2, scales, out_host, ws, stream=None,
+                      check=True) -> int:
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _host_io(ctypes.byref(dims), _ptr(x_host), _ptr(router_w), _ptr(w13), _ptr(w2), sp,
+                  _ptr(out_host), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_host_io") if check else st
+
+
+def fused_moe_get_device_status(ws, stream=None) -> int:
+    return int(_dev_status(_ptr(ws), _stream(stream)))
+
+
+def fused_moe_debug_scalars(ws, stream=None):
+    """({amax_x, s1, inv1, amax_h, s2, inv2}, {n_chunks, split1, split2})."""
+    f = (c_float * 6)()
+    i = (c_int32 * 3)()
+    _check(_dbg(_ptr(ws), f, i, _stream(stream)), "fused_moe_debug_scalars")
+    names_f = ("amax_x", "s1", "inv1", "amax_h", "s2", "inv2")
+    names_i = ("n_chunks", "split1", "split2")
+    return dict(zip(names_f, list(f))), dict(zip(names_i, list(i)))
+
+
+def fused_moe_launches_per_call(dims) -> int:
+    return int(_launches(ctypes.byref(dims)))
+
+
+def fused_moe_profile(dims, x, router_w, w13, w2, scales, out, ws, stream=None):
+    """One fused_moe call with an event after every launch: [(kernel name, ms), ...]."""
+    cap = 32
+    ms = (c_float * cap)()
+    names = (c_char_p * cap)()
+    n = c_int32(0)
+    sp = ctypes.byref(scales) if scales is not None else None
+    _check(_profile(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(w13), _ptr(w2), sp,
+                    _ptr(out), _ptr(ws), ws.numel(), _stream(stream), ms, names, cap,
+                    ctypes.byref(n)), "fused_moe_profile")
+    return [(names[i].decode(), float(ms[i])) for i in range(n.value)]
+
+
+class FusedMoE:
+    """The whole layer on device tensors, with its own workspace.
+
+    x [T,H] bf16, router_w [E,H] bf16, w13 [E,2I,H] and w2 [E,H,I] as uint8 e4m3
+    bytes (with w13_scale, w2_scale [E] fp32) or bf16.  Returns out [T,H] bf16."""
+
+    def __init__(self, router_w, w13, w2, top_k, w13_scale=None, w2_scale=None,
+                 a1_scale=0.0, a2_scale=0.0, variant="auto"):
+        self.router_w, self.w13, self.w2 = router_w, w13, w2
+        self.top_k, self.variant = top_k, variant
+        self.w13_scale, self.w2_scale = w13_scale, w2_scale
+        self.scales = make_scales(w13_scale, w2_scale, a1_scale, a2_scale)
+        self._ws = {}
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if T not in self._ws:
+            dims = make_dims(T, self.w13.shape[2], self.w13.shape[1] // 2, self.w13.shape[0],
+                             self.top_k, self.w13.dtype == torch.uint8, self.variant)
+            self._ws[T] = alloc_workspace(dims, self.w13.device)
+        return self._ws[T]
+
+    def dims(self, T: int) -> FmoeDims:
+        return make_dims(T, self.w13.shape[2], self.w13.shape[1] // 2, self.w13.shape[0],
+                         self.top_k, self.w13.dtype == torch.uint8, self.variant)
+
+    def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty(T, x.shape[1], dtype=torch.bfloat16, device=x.device)
+        fused_moe(self.dims(T), x, self.router_w, self.w13, self.w2, self.scales, out,
+                  self.workspace(T), stream)
+        return out

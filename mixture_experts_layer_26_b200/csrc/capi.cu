@@ -1,0 +1,597 @@
+// Host side of the C ABI declared in include/fused_moe.h: argument checks, workspace
+// layout, TMA descriptors and the launch sequence of each step.  Nothing here
+// allocates device memory or synchronises, except the calls the header documents as
+// synchronous.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fmoe_kernels.h"
+#include "fused_moe.h"
+
+using namespace fmoe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kPartialBudget = size_t(64) << 20;  // bytes of split-K partials per GEMM
+constexpr int kMaxSplit = 16;
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // bounded mbarrier waits: 2 s
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+  bool fp8 = false, swap = false;
+  int R = 0, chunk_rows = 0, max_chunks = 0, s1max = 0, s2max = 0;
+  size_t hdr = 0, amax_x = 0, amax_h = 0, chunks = 0;
+  size_t ids = 0, tw = 0, counts = 0, offsets = 0, rows = 0, inv = 0;
+  size_t x_in = 0, out_dev = 0, a_perm = 0, p1 = 0, h = 0, hq = 0, p2 = 0, y = 0;
+  size_t total = 0;
+};
+
+fmoe_status check_dims(const fmoe_dims* d) {
+  if (d == nullptr) return FMOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->H < 1 || d->I < 1 || d->E < 1 || d->E > kMaxExperts || d->top_k < 1 ||
+      d->top_k > d->E)
+    return FMOE_ERR_INVALID_ARG;
+  if (d->wdtype != FMOE_BF16 && d->wdtype != FMOE_FP8_E4M3) return FMOE_ERR_INVALID_ARG;
+  if (d->variant < FMOE_VARIANT_AUTO || d->variant > FMOE_VARIANT_NORMAL)
+    return FMOE_ERR_INVALID_ARG;
+  if (d->H % 256 != 0 || d->I % 128 != 0 || d->H > 16384) return FMOE_ERR_UNSUPPORTED;
+  const int64_t R = static_cast<int64_t>(d->T) * d->top_k;
+  const int64_t lim = int64_t(1) << 31;
+  if (R * std::max<int64_t>(d->H, 2 * int64_t(d->I)) >= lim) return FMOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->E) * 2 * d->I >= lim || static_cast<int64_t>(d->E) * d->H >= lim)
+    return FMOE_ERR_UNSUPPORTED;
+  return FMOE_OK;
+}
+
+Layout make_layout(const fmoe_dims& d) {
+  Layout L;
+  L.fp8 = d.wdtype == FMOE_FP8_E4M3;
+  const int T = d.T, H = d.H, I = d.I, E = d.E;
+  const int R = T * d.top_k;
+  L.R = R;
+  int variant = d.variant;
+  if (variant == FMOE_VARIANT_AUTO)
+    variant = ((R + E - 1) / E <= 64) ? FMOE_VARIANT_SWAP_AB : FMOE_VARIANT_NORMAL;
+  L.swap = variant == FMOE_VARIANT_SWAP_AB;
+  // an expert receives at most T rows (one per token)
+  L.chunk_rows = L.swap ? std::min(64, static_cast<int>(align_up(std::max(T, 1), 16))) : 128;
+  L.max_chunks = R / L.chunk_rows + std::min(E, R) + 1;
+  const size_t es = L.fp8 ? 1 : 2;
+  const size_t p1_plane = static_cast<size_t>(R) * 2 * I * 4;
+  const size_t p2_plane = static_cast<size_t>(R) * H * 4;
+  if (L.swap) {
+    L.s1max = static_cast<int>(std::clamp<size_t>(kPartialBudget / std::max<size_t>(p1_plane, 1), 1, kMaxSplit));
+    L.s2max = static_cast<int>(std::clamp<size_t>(kPartialBudget / std::max<size_t>(p2_plane, 1), 1, kMaxSplit));
+  }
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L.hdr = take(sizeof(WsHeader));
+  L.amax_x = take(static_cast<size_t>(std::max(T, 1)) * 4);
+  L.amax_h = take(static_cast<size_t>(kAmaxSlots) * 4);
+  L.chunks = take(static_cast<size_t>(L.max_chunks) * sizeof(Chunk));
+  L.ids = take(static_cast<size_t>(R) * 4);
+  L.tw = take(static_cast<size_t>(R) * 4);
+  L.counts = take(static_cast<size_t>(E) * 4);
+  L.offsets = take(static_cast<size_t>(E + 1) * 4);
+  L.rows = take(static_cast<size_t>(R) * 4);
+  L.inv = take(static_cast<size_t>(R) * 4);
+  L.x_in = take(static_cast<size_t>(T) * H * 2);
+  L.out_dev = take(static_cast<size_t>(T) * H * 2);
+  L.a_perm = take(static_cast<size_t>(R) * H * es);
+  L.p1 = take(L.swap ? L.s1max * p1_plane : 0);
+  L.h = take(L.fp8 ? static_cast<size_t>(R) * I * 4 : 0);
+  L.hq = take(static_cast<size_t>(R) * I * es);
+  L.p2 = take(L.swap ? L.s2max * p2_plane : 0);
+  L.y = take(static_cast<size_t>(R) * H * 4);
+  L.total = off;
+  return L;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fmoe_status check_ws(const Layout& L, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return FMOE_ERR_WORKSPACE;
+  if (ws_bytes < L.total) return FMOE_ERR_WORKSPACE;
+  return FMOE_OK;
+}
+
+// Every pointer non-null and 16-byte aligned.
+template <typename... P>
+fmoe_status check_ptrs(P... ptrs) {
+  const void* list[] = {static_cast<const void*>(ptrs)...};
+  for (const void* p : list) {
+    if (p == nullptr) return FMOE_ERR_INVALID_ARG;
+    if (!aligned16(p)) return FMOE_ERR_UNSUPPORTED;
+  }
+  return FMOE_OK;
+}
+
+fmoe_status check_fp8_scales(const fmoe_dims& d, const fmoe_scales* sc) {
+  if (d.wdtype != FMOE_FP8_E4M3) return FMOE_OK;
+  if (sc == nullptr || sc->w13_scale == nullptr || sc->w2_scale == nullptr)
+    return FMOE_ERR_INVALID_ARG;
+  return FMOE_OK;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D K-major operand [rows, inner] with 128-byte rows per box and the 128-byte swizzle.
+bool encode_map(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows,
+                uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tma_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline fmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA; }
+
+#define FMOE_TRY(expr)                   \
+  do {                                   \
+    const fmoe_status _s = (expr);       \
+    if (_s != FMOE_OK) return _s;        \
+  } while (0)
+
+// Measurement hook: when active (fused_moe_profile only), every kernel launch of the
+// call sequence is followed by an event record on the launching stream.
+struct StageRecorder {
+  static constexpr int kCap = 32;
+  bool active = false;
+  int n = 0;
+  cudaEvent_t ev[kCap + 1] = {};
+  const char* names[kCap] = {};
+};
+thread_local StageRecorder g_rec;
+
+inline cudaError_t mark(const char* name, cudaStream_t s) {
+  if (!g_rec.active) return cudaSuccess;
+  if (g_rec.n >= StageRecorder::kCap) return cudaSuccess;
+  g_rec.names[g_rec.n] = name;
+  return cudaEventRecord(g_rec.ev[++g_rec.n], s);
+}
+
+// launch `expr` (a launcher returning cudaError_t), then mark it
+#define FMOE_LAUNCH(name, expr, stream)                      \
+  do {                                                       \
+    FMOE_TRY(cuda_status(expr));                             \
+    FMOE_TRY(cuda_status(mark(name, stream)));               \
+  } while (0)
+
+
+// ------------------------------------------------------------------ step bodies
+
+fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
+                       int32_t* ids, float* tw, char* W, cudaStream_t s) {
+  RouterArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.wr = static_cast<const uint16_t*>(rw);
+  a.topk_ids = ids;
+  a.topk_w = tw;
+  a.amax_part = reinterpret_cast<float*>(W + L.amax_x);
+  a.hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+  a.T = d.T;
+  a.H = d.H;
+  a.E = d.E;
+  a.k = d.top_k;
+  a.num_sms = num_sms();
+  FMOE_LAUNCH("router", launch_router(a, s), s);
+  return FMOE_OK;
+}
+
+fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids, const void* x,
+                         const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
+                         int32_t* inv, void* a_perm, char* W, cudaStream_t s) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+  PermuteArgs p{};
+  p.topk_ids = ids;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.sorted_rows = rows;
+  p.inv_perm = inv;
+  p.amax_part = reinterpret_cast<const float*>(W + L.amax_x);
+  p.hdr = hdr;
+  p.R = L.R;
+  p.E = d.E;
+  p.k = d.top_k;
+  p.fp8 = L.fp8 ? 1 : 0;
+  p.a1_static = sc != nullptr ? sc->a1_scale : 0.f;
+  FMOE_LAUNCH("permute", launch_permute(p, s), s);
+  GatherArgs g{};
+  g.x = static_cast<const uint16_t*>(x);
+  g.sorted_rows = rows;
+  g.a_perm = a_perm;
+  g.hdr = hdr;
+  g.status = &hdr->status;
+  g.R = L.R;
+  g.H = d.H;
+  g.k = d.top_k;
+  g.fp8 = p.fp8;
+  FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
+  return FMOE_OK;
+}
+
+fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm,
+                         const int32_t* offsets, const int32_t* rows, const float* tw,
+                         const void* w13, const void* w2, const fmoe_scales* sc, float* y,
+                         char* W, cudaStream_t s) {
+  const int sms = num_sms();
+  const bool fp8 = L.fp8, swap = L.swap;
+  const int H = d.H, I = d.I, E = d.E, R = L.R;
+  const int bk = fp8 ? 128 : 64;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+  Chunk* chunks = reinterpret_cast<Chunk*>(W + L.chunks);
+  float* amax_h = reinterpret_cast<float*>(W + L.amax_h);
+  float* hbuf = reinterpret_cast<float*>(W + L.h);
+  void* hq = W + L.hq;
+
+  PlanArgs pa{};
+  pa.offsets = offsets;
+  pa.chunks = chunks;
+  pa.hdr = hdr;
+  pa.R = R;
+  pa.E = E;
+  pa.chunk_rows = L.chunk_rows;
+  pa.max_chunks = L.max_chunks;
+  pa.swap_ab = swap ? 1 : 0;
+  pa.units1_per_chunk = swap ? 2 * I / 128 : I / 128;
+  pa.units2_per_chunk = swap ? H / 128 : H / 256;
+  pa.kblocks1 = H / bk;
+  pa.kblocks2 = I / bk;
+  pa.s1max = std::max(L.s1max, 1);
+  pa.s2max = std::max(L.s2max, 1);
+  pa.num_sms = sms;
+  FMOE_LAUNCH("plan", launch_plan(pa, s), s);
+
+  const uint32_t xbox = swap ? 16u : 128u;
+  GemmArgs g{};
+  if (!encode_map(&g.map_w, w13, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(E) * 2 * I, 128) ||
+      !encode_map(&g.map_x, a_perm, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(R), xbox))
+    return FMOE_ERR_CUDA;
+  g.chunks = chunks;
+  g.hdr = hdr;
+  g.hdr_w = hdr;
+  g.status = &hdr->status;
+  g.out = swap ? reinterpret_cast<float*>(W + L.p1) : (fp8 ? hbuf : nullptr);
+  g.out_bf16 = (!swap && !fp8) ? static_cast<uint16_t*>(hq) : nullptr;
+  g.w_scale = fp8 ? sc->w13_scale : nullptr;
+  g.topk_w = tw;
+  g.sorted_rows = rows;
+  g.amax_part = amax_h;
+  g.R = R;
+  g.K = H;
+  g.Nout = 2 * I;
+  g.I = I;
+  g.H = H;
+  g.rows_per_expert = 2 * I;
+  g.chunk_rows = L.chunk_rows;
+  g.nstages = gemm_stages(swap, L.chunk_rows);
+  g.wait_budget_ns = kWaitBudgetNs;
+  FMOE_LAUNCH(swap ? "gemm1_swapab" : "gemm1_normal", launch_gemm(g, fp8, swap, 1, sms, s), s);
+
+  if (swap) {
+    Finalize1Args f{};
+    f.part = reinterpret_cast<const float*>(W + L.p1);
+    f.offsets = offsets;
+    f.w13_scale = fp8 ? sc->w13_scale : nullptr;
+    f.h = fp8 ? hbuf : nullptr;
+    f.hq_bf16 = fp8 ? nullptr : static_cast<uint16_t*>(hq);
+    f.amax_part = amax_h;
+    f.hdr = hdr;
+    f.R = R;
+    f.I = I;
+    f.E = E;
+    f.fp8 = fp8 ? 1 : 0;
+    FMOE_LAUNCH("finalize1", launch_finalize1(f, sms, s), s);
+  }
+  if (fp8) {
+    QuantHArgs q{};
+    q.h = hbuf;
+    q.hq = static_cast<uint8_t*>(hq);
+    q.amax_part = amax_h;
+    q.hdr = hdr;
+    q.R = R;
+    q.I = I;
+    q.a2_static = sc != nullptr ? sc->a2_scale : 0.f;
+    FMOE_LAUNCH("quant_h", launch_quant_h(q, sms, s), s);
+  }
+
+  GemmArgs g2 = g;
+  if (!encode_map(&g2.map_w, w2, fp8, static_cast<uint64_t>(I), static_cast<uint64_t>(E) * H, 128) ||
+      !encode_map(&g2.map_x, hq, fp8, static_cast<uint64_t>(I), static_cast<uint64_t>(R), xbox))
+    return FMOE_ERR_CUDA;
+  g2.out = swap ? reinterpret_cast<float*>(W + L.p2) : y;
+  g2.out_bf16 = nullptr;
+  g2.w_scale = fp8 ? sc->w2_scale : nullptr;
+  g2.K = I;
+  g2.Nout = H;
+  g2.rows_per_expert = H;
+  FMOE_LAUNCH(swap ? "gemm2_swapab" : "gemm2_normal", launch_gemm(g2, fp8, swap, 2, sms, s), s);
+
+  if (swap) {
+    Finalize2Args f{};
+    f.part = reinterpret_cast<const float*>(W + L.p2);
+    f.offsets = offsets;
+    f.w2_scale = fp8 ? sc->w2_scale : nullptr;
+    f.topk_w = tw;
+    f.sorted_rows = rows;
+    f.hdr = hdr;
+    f.status = &hdr->status;
+    f.y = y;
+    f.R = R;
+    f.H = H;
+    f.E = E;
+    f.fp8 = fp8 ? 1 : 0;
+    FMOE_LAUNCH("finalize2", launch_finalize2(f, sms, s), s);
+  }
+  return FMOE_OK;
+}
+
+fmoe_status combine_impl(const fmoe_dims& d, const float* y, const int32_t* inv, void* out,
+                         cudaStream_t s) {
+  CombineArgs c{};
+  c.y = y;
+  c.inv_perm = inv;
+  c.out = static_cast<uint16_t*>(out);
+  c.T = d.T;
+  c.H = d.H;
+  c.k = d.top_k;
+  FMOE_LAUNCH("combine", launch_combine(c, num_sms(), s), s);
+  return FMOE_OK;
+}
+
+fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
+                       const void* w13, const void* w2, const fmoe_scales* sc, void* out, char* W,
+                       cudaStream_t s) {
+  int32_t* ids = reinterpret_cast<int32_t*>(W + L.ids);
+  float* tw = reinterpret_cast<float*>(W + L.tw);
+  int32_t* counts = reinterpret_cast<int32_t*>(W + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(W + L.offsets);
+  int32_t* rows = reinterpret_cast<int32_t*>(W + L.rows);
+  int32_t* inv = reinterpret_cast<int32_t*>(W + L.inv);
+  float* y = reinterpret_cast<float*>(W + L.y);
+  FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
+  FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s));
+  FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s));
+  return combine_impl(d, y, inv, out, s);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ public API
+
+extern "C" {
+
+int32_t fused_moe_abi_version(void) { return FUSED_MOE_ABI_VERSION; }
+
+const char* fused_moe_status_string(fmoe_status st) {
+  switch (st) {
+    case FMOE_OK: return "FMOE_OK";
+    case FMOE_ERR_INVALID_ARG: return "FMOE_ERR_INVALID_ARG";
+    case FMOE_ERR_UNSUPPORTED: return "FMOE_ERR_UNSUPPORTED";
+    case FMOE_ERR_WORKSPACE: return "FMOE_ERR_WORKSPACE";
+    case FMOE_ERR_CUDA: return "FMOE_ERR_CUDA";
+    case FMOE_ERR_TIMEOUT: return "FMOE_ERR_TIMEOUT";
+    case FMOE_ERR_DEVICE_BOUNDS: return "FMOE_ERR_DEVICE_BOUNDS";
+  }
+  return "FMOE_ERR_UNKNOWN";
+}
+
+size_t fused_moe_workspace_size(const fmoe_dims* dims) {
+  if (check_dims(dims) != FMOE_OK) return 0;
+  return make_layout(*dims).total;
+}
+
+fmoe_status fused_moe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream stream) {
+  if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
+  if (ws_bytes < sizeof(WsHeader)) return FMOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+}
+
+fmoe_status fused_moe_route(const fmoe_dims* dims, const void* x, const void* router_w,
+                            int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                            fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, router_w, topk_ids, topk_w));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  return route_impl(*dims, L, x, router_w, topk_ids, topk_w, static_cast<char*>(ws),
+                    static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_permute(const fmoe_dims* dims, const int32_t* topk_ids, const void* x,
+                              const fmoe_scales* scales, int32_t* counts, int32_t* offsets,
+                              int32_t* sorted_rows, int32_t* inv_perm, void* a_perm, void* ws,
+                              size_t ws_bytes, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(topk_ids, x, counts, offsets, sorted_rows, inv_perm, a_perm));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  return permute_impl(*dims, L, topk_ids, x, scales, counts, offsets, sorted_rows, inv_perm,
+                      a_perm, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_experts(const fmoe_dims* dims, const void* a_perm, const int32_t* offsets,
+                              const int32_t* sorted_rows, const float* topk_w, const void* w13,
+                              const void* w2, const fmoe_scales* scales, float* y_perm, void* ws,
+                              size_t ws_bytes, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(a_perm, offsets, sorted_rows, topk_w, w13, w2, y_perm));
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  return experts_impl(*dims, L, a_perm, offsets, sorted_rows, topk_w, w13, w2, scales, y_perm,
+                      static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_combine(const fmoe_dims* dims, const float* y_perm, const int32_t* inv_perm,
+                              void* out, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(y_perm, inv_perm, out));
+  return combine_impl(*dims, y_perm, inv_perm, out, static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe(const fmoe_dims* dims, const void* x, const void* router_w, const void* w13,
+                      const void* w2, const fmoe_scales* scales, void* out, void* ws,
+                      size_t ws_bytes, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, router_w, w13, w2, out));
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  return fused_impl(*dims, L, x, router_w, w13, w2, scales, out, static_cast<char*>(ws),
+                    static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host, const void* router_w,
+                              const void* w13, const void* w2, const fmoe_scales* scales,
+                              void* out_host, void* ws, size_t ws_bytes, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  if (x_host == nullptr || out_host == nullptr) return FMOE_ERR_INVALID_ARG;
+  FMOE_TRY(check_ptrs(router_w, w13, w2));
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  char* W = static_cast<char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xbytes = static_cast<size_t>(dims->T) * dims->H * 2;
+  FMOE_TRY(cuda_status(cudaMemcpyAsync(W + L.x_in, x_host, xbytes, cudaMemcpyHostToDevice, s)));
+  FMOE_TRY(fused_impl(*dims, L, W + L.x_in, router_w, w13, w2, scales, W + L.out_dev, W, s));
+  FMOE_TRY(cuda_status(cudaMemcpyAsync(out_host, W + L.out_dev, xbytes, cudaMemcpyDeviceToHost, s)));
+  return cuda_status(cudaStreamSynchronize(s));
+}
+
+int32_t fused_moe_launches_per_call(const fmoe_dims* dims) {
+  if (check_dims(dims) != FMOE_OK) return -1;
+  if (dims->T == 0) return 0;
+  const Layout L = make_layout(*dims);
+  // router, permute, gather, plan, gemm1, [finalize1], [quant_h], gemm2, [finalize2], combine
+  return 7 + (L.swap ? 2 : 0) + (L.fp8 ? 1 : 0);
+}
+
+fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, const void* router_w,
+                              const void* w13, const void* w2, const fmoe_scales* scales, void* out,
+                              void* ws, size_t ws_bytes, fmoe_stream stream, float* ms_host,
+                              const char** names_host, int32_t cap, int32_t* n_host) {
+  FMOE_TRY(check_dims(dims));
+  if (n_host == nullptr || ms_host == nullptr || cap < 1) return FMOE_ERR_INVALID_ARG;
+  *n_host = 0;
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, router_w, w13, w2, out));
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local bool created = false;
+  if (!created) {
+    for (auto& e : g_rec.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return FMOE_ERR_CUDA;
+    created = true;
+  }
+  g_rec.n = 0;
+  g_rec.active = true;
+  fmoe_status st = cuda_status(cudaEventRecord(g_rec.ev[0], s));
+  if (st == FMOE_OK)
+    st = fused_impl(*dims, L, x, router_w, w13, w2, scales, out, static_cast<char*>(ws), s);
+  g_rec.active = false;
+  FMOE_TRY(st);
+  FMOE_TRY(cuda_status(cudaStreamSynchronize(s)));
+  const int n = std::min<int>(g_rec.n, cap);
+  for (int i = 0; i < n; ++i) {
+    float ms = 0.f;
+    FMOE_TRY(cuda_status(cudaEventElapsedTime(&ms, g_rec.ev[i], g_rec.ev[i + 1])));
+    ms_host[i] = ms;
+    if (names_host != nullptr) names_host[i] = g_rec.names[i];
+  }
+  *n_host = n;
+  return FMOE_OK;
+}
+
+fmoe_status fused_moe_get_device_status(const void* ws, fmoe_stream stream) {
+  if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
+  int32_t st = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&st, ws, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return FMOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FMOE_ERR_CUDA;
+  return static_cast<fmoe_status>(st);
+}
+
+fmoe_status fused_moe_debug_scalars(const void* ws, float* f6, int32_t* i3, fmoe_stream stream) {
+  if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
+  WsHeader h;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (f6 != nullptr) {
+    f6[0] = h.amax_x;
+    f6[1] = h.s1;
+    f6[2] = h.inv1;
+    f6[3] = h.amax_h;
+    f6[4] = h.s2;
+    f6[5] = h.inv2;
+  }
+  if (i3 != nullptr) {
+    i3[0] = h.n_chunks;
+    i3[1] = h.split1;
+    i3[2] = h.split2;
+  }
+  return FMOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,244 @@
+// Element-wise steps around the grouped GEMMs.
+//
+// finalize1: sum the split-K partials of the first contraction, apply the scale
+//   s1*sw13[e], h = SiLU(g)*u (gate = rows 0..I-1 of w13, up = rows I..2I-1), and keep a
+//   per-CTA max |h|.  FP8 format: h stays fp32 for the second quantisation.  bf16
+//   format: h is rounded to bf16 and is already the second GEMM's input.
+// quant_h: reduce the max |h| partials into the per-tensor scale s2 = amax/448 (or a
+//   static scale), then hq = e4m3(h * 448/amax) rounded to nearest even, saturating.
+// finalize2: sum the split-K partials of the second contraction, apply s2*sw2[e] and
+//   the routing weight of the row.
+// combine: out[t] = bf16( sum over j < k of y[inv_perm[t*k+j]] ), fp32 adds in j order
+//   ("expert aggregation", codebridge-ai.com blog on the AWS MoE kernels,
+//   "2. Backend routing: Triton over CUTLASS").
+//
+// All four are HBM/L2-bound and use 16-byte vector accesses; their grids are a
+// multiple of the SM count.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "fmoe_kernels.h"
+
+namespace fmoe {
+
+namespace {
+
+constexpr int kEwThreads = 256;
+
+__device__ __forceinline__ int expert_of_row(const int* offs, int E, int p) {
+  // largest e with offs[e] <= p (offsets are non-decreasing; empty experts repeat)
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offs[mid] <= p) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = 0.f;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < kEwThreads / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize1_kernel(Finalize1Args a) {
+  __shared__ int offs[kMaxExperts + 1];
+  __shared__ float red[kEwThreads / 32];
+  for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];
+  __syncthreads();
+  const int S = a.hdr->split1;
+  const float s1 = a.fp8 ? a.hdr->s1 : 1.f;
+  const int I = a.I, I4 = a.I / 4;
+  const size_t plane = static_cast<size_t>(a.R) * 2 * I;
+  const size_t total = static_cast<size_t>(a.R) * I4;
+  float amax = 0.f;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const int p = static_cast<int>(idx / I4), c = static_cast<int>(idx % I4) * 4;
+    const int e = expert_of_row(offs, a.E, p);
+    const float sc = a.fp8 ? s1 * a.w13_scale[e] : 1.f;
+    const float* gp = a.part + static_cast<size_t>(p) * 2 * I + c;
+    float4 g = *reinterpret_cast<const float4*>(gp);
+    float4 u = *reinterpret_cast<const float4*>(gp + I);
+    for (int s = 1; s < S; ++s) {
+      const float4 g2 = *reinterpret_cast<const float4*>(gp + s * plane);
+      const float4 u2 = *reinterpret_cast<const float4*>(gp + s * plane + I);
+      g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+      u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+    }
+    float4 h;
+    h.x = silu_f(g.x * sc) * (u.x * sc);
+    h.y = silu_f(g.y * sc) * (u.y * sc);
+    h.z = silu_f(g.z * sc) * (u.z * sc);
+    h.w = silu_f(g.w * sc) * (u.w * sc);
+    const size_t o = static_cast<size_t>(p) * I + c;
+    if (a.fp8) {
+      *reinterpret_cast<float4*>(a.h + o) = h;
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w))));
+    } else {
+      const __nv_bfloat162 b0 = __floats2bfloat162_rn(h.x, h.y);
+      const __nv_bfloat162 b1 = __floats2bfloat162_rn(h.z, h.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&b0);
+      pk.y = *reinterpret_cast<const uint32_t*>(&b1);
+      *reinterpret_cast<uint2*>(a.hq_bf16 + o) = pk;
+    }
+  }
+  const float m = block_max(amax, red);
+  if (threadIdx.x == 0) {
+    a.amax_part[blockIdx.x] = m;
+    if (blockIdx.x == 0) a.hdr->amax_h_count = gridDim.x;
+  }
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+__global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
+  __shared__ float s_inv;
+  if (threadIdx.x < 32) {
+    float m = 0.f;
+    const int n = a.hdr->amax_h_count;
+    for (int i = threadIdx.x; i < n; i += 32) m = fmaxf(m, a.amax_part[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (threadIdx.x == 0) {
+      float s2 = 1.f, inv2 = 1.f;
+      if (a.a2_static > 0.f) {
+        s2 = a.a2_static;
+        inv2 = 1.0f / a.a2_static;
+      } else if (m > 0.f) {
+        s2 = m / 448.0f;
+        inv2 = 448.0f / m;
+      }
+      s_inv = inv2;
+      if (blockIdx.x == 0) {
+        a.hdr->amax_h = m;
+        a.hdr->s2 = s2;
+        a.hdr->inv2 = inv2;
+      }
+    }
+  }
+  __syncthreads();
+  const float inv = s_inv;
+  const size_t total = static_cast<size_t>(a.R) * a.I / 16;
+  for (size_t v = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; v < total;
+       v += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const float4* src = reinterpret_cast<const float4*>(a.h) + 4 * v;
+    const float4 f0 = src[0], f1 = src[1], f2 = src[2], f3 = src[3];
+    uint4 q;
+    q.x = e4m3x4(f0.x * inv, f0.y * inv, f0.z * inv, f0.w * inv);
+    q.y = e4m3x4(f1.x * inv, f1.y * inv, f1.z * inv, f1.w * inv);
+    q.z = e4m3x4(f2.x * inv, f2.y * inv, f2.z * inv, f2.w * inv);
+    q.w = e4m3x4(f3.x * inv, f3.y * inv, f3.z * inv, f3.w * inv);
+    reinterpret_cast<uint4*>(a.hq)[v] = q;
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize2_kernel(Finalize2Args a) {
+  __shared__ int offs[kMaxExperts + 1];
+  for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];
+  __syncthreads();
+  const int S = a.hdr->split2;
+  const float s2 = a.fp8 ? a.hdr->s2 : 1.f;
+  const int H = a.H, H4 = a.H / 4;
+  const size_t plane = static_cast<size_t>(a.R) * H;
+  const size_t total = static_cast<size_t>(a.R) * H4;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const int p = static_cast<int>(idx / H4), c = static_cast<int>(idx % H4) * 4;
+    const int e = expert_of_row(offs, a.E, p);
+    const float sc = a.fp8 ? s2 * a.w2_scale[e] : 1.f;
+    const int src_row = a.sorted_rows[p];
+    if (src_row < 0 || src_row >= a.R) {
+      record_status(a.status, ST_BOUNDS);
+      continue;
+    }
+    const float wr = a.topk_w[src_row];
+    const float* src = a.part + static_cast<size_t>(p) * H + c;
+    float4 v = *reinterpret_cast<const float4*>(src);
+    for (int s = 1; s < S; ++s) {
+      const float4 v2 = *reinterpret_cast<const float4*>(src + s * plane);
+      v.x += v2.x; v.y += v2.y; v.z += v2.z; v.w += v2.w;
+    }
+    v.x = v.x * sc * wr;
+    v.y = v.y * sc * wr;
+    v.z = v.z * sc * wr;
+    v.w = v.w * sc * wr;
+    *reinterpret_cast<float4*>(a.y + static_cast<size_t>(p) * H + c) = v;
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) combine_kernel(CombineArgs a) {
+  const int H8 = a.H / 8;
+  const size_t total = static_cast<size_t>(a.T) * H8;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const int t = static_cast<int>(idx / H8), c = static_cast<int>(idx % H8) * 8;
+    float acc[8];
+    for (int j = 0; j < a.k; ++j) {
+      int p = a.inv_perm[static_cast<size_t>(t) * a.k + j];
+      if (p < 0 || p >= a.T * a.k) p = 0;  // malformed permutation: stay in bounds
+      const float4* src = reinterpret_cast<const float4*>(a.y + static_cast<size_t>(p) * a.H + c);
+      const float4 v0 = src[0], v1 = src[1];
+      if (j == 0) {
+        acc[0] = v0.x; acc[1] = v0.y; acc[2] = v0.z; acc[3] = v0.w;
+        acc[4] = v1.x; acc[5] = v1.y; acc[6] = v1.z; acc[7] = v1.w;
+      } else {
+        acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+        acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+      }
+    }
+    uint4 o;
+    __nv_bfloat162 b;
+    b = __floats2bfloat162_rn(acc[0], acc[1]); o.x = *reinterpret_cast<uint32_t*>(&b);
+    b = __floats2bfloat162_rn(acc[2], acc[3]); o.y = *reinterpret_cast<uint32_t*>(&b);
+    b = __floats2bfloat162_rn(acc[4], acc[5]); o.z = *reinterpret_cast<uint32_t*>(&b);
+    b = __floats2bfloat162_rn(acc[6], acc[7]); o.w = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = o;
+  }
+}
+
+int ew_grid(size_t work_items, int num_sms) {
+  const size_t per_cta = kEwThreads;
+  size_t g = (work_items + per_cta - 1) / per_cta;
+  const size_t cap = static_cast<size_t>(num_sms) * 8;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_finalize1(const Finalize1Args& a, int num_sms, cudaStream_t s) {
+  int grid = ew_grid(static_cast<size_t>(a.R) * a.I / 4, num_sms);
+  if (grid > kAmaxSlots) grid = kAmaxSlots;
+  finalize1_kernel<<<grid, kEwThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_h(const QuantHArgs& a, int num_sms, cudaStream_t s) {
+  quant_h_kernel<<<ew_grid(static_cast<size_t>(a.R) * a.I / 16, num_sms), kEwThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize2(const Finalize2Args& a, int num_sms, cudaStream_t s) {
+  finalize2_kernel<<<ew_grid(static_cast<size_t>(a.R) * a.H / 4, num_sms), kEwThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
+  combine_kernel<<<ew_grid(static_cast<size_t>(a.T) * a.H / 8, num_sms), kEwThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fmoe

@@ -1,0 +1,151 @@
+// Internal launcher interface between the C ABI (capi.cu) and the kernel files.
+// Every launcher enqueues work on `stream` and returns cudaGetLastError().
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fmoe_common.cuh"
+
+namespace fmoe {
+
+// Raise a kernel's dynamic shared memory limit once per device (one bit mask per kernel).
+template <auto Kernel>
+inline cudaError_t set_max_dynamic_smem(int bytes) {
+  static unsigned configured = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const unsigned bit = 1u << (dev & 31);
+  if (configured & bit) return cudaSuccess;
+  err = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) configured |= bit;
+  return err;
+}
+
+// ----------------------------------------------------------------------------- router
+struct RouterArgs {
+  const uint16_t* x;    // [T, H] bf16 bits
+  const uint16_t* wr;   // [E, H] bf16 bits
+  int32_t* topk_ids;    // [T, k]
+  float* topk_w;        // [T, k]
+  float* amax_part;     // [ceil(T / tokens_per_cta)] per-CTA max |x|
+  WsHeader* hdr;
+  int T, H, E, k;
+  int num_sms;
+};
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+int router_tokens_per_cta(int T, int H, int E, int num_sms);
+
+// ----------------------------------------------------------------------------- permute
+struct PermuteArgs {
+  const int32_t* topk_ids;  // [R]
+  int32_t* counts;          // [E]
+  int32_t* offsets;         // [E + 1]
+  int32_t* sorted_rows;     // [R]
+  int32_t* inv_perm;        // [R]
+  const float* amax_part;   // router partials
+  WsHeader* hdr;
+  int R, E, k;
+  int fp8;                  // compute the activation scale (FP8 format)
+  float a1_static;          // > 0: static scale
+};
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+
+struct GatherArgs {
+  const uint16_t* x;          // [T, H] bf16
+  const int32_t* sorted_rows; // [R]
+  void* a_perm;               // [R, H] e4m3 bytes or bf16
+  const WsHeader* hdr;        // inv1
+  int32_t* status;
+  int R, H, k;
+  int fp8;
+};
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- experts
+struct PlanArgs {
+  const int32_t* offsets;  // [E + 1]
+  Chunk* chunks;           // [max_chunks]
+  WsHeader* hdr;
+  int R, E, chunk_rows, max_chunks;
+  int swap_ab;
+  int units1_per_chunk;    // output tiles of the first contraction per chunk
+  int units2_per_chunk;
+  int kblocks1, kblocks2;  // K blocks of each contraction
+  int s1max, s2max;        // largest split-K factors the workspace holds
+  int num_sms;
+};
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
+
+struct GemmArgs {
+  CUtensorMap map_w;       // weights [E * rows_per_expert, K], box {BK, 128}
+  CUtensorMap map_x;       // activations [R, K], box {BK, 16 (swap) or 128 (normal)}
+  const Chunk* chunks;
+  const WsHeader* hdr;
+  int32_t* status;
+  float* out;              // swap: partials [S][R][Nout]; normal: h [R, I] or y [R, H]
+  uint16_t* out_bf16;      // normal, first contraction, bf16 format: h rounded to bf16
+  const float* w_scale;    // [E] per-expert weight scale (FP8) or null
+  const float* topk_w;     // [R] flattened routing weights (normal, second contraction)
+  const int32_t* sorted_rows;
+  float* amax_part;        // normal, first contraction: per-CTA max |h|
+  WsHeader* hdr_w;         // amax_h_count (normal, first contraction)
+  int R, K, Nout, I, H;
+  int rows_per_expert;     // weight rows per expert in map_w (2I or H)
+  int chunk_rows;
+  int nstages;             // shared-memory pipeline depth (gemm_stages)
+  uint64_t wait_budget_ns;
+};
+// gemm = 1 (w13, gate/up) or 2 (w2); fp8 selects kind::f8f6f4 vs kind::f16.
+cudaError_t launch_gemm(const GemmArgs& a, bool fp8, bool swap_ab, int gemm, int num_sms,
+                        cudaStream_t s);
+int gemm_stages(bool swap_ab, int chunk_rows);
+
+struct Finalize1Args {
+  const float* part;        // [S][R][2I]
+  const int32_t* offsets;   // [E + 1]
+  const float* w13_scale;   // [E] or null
+  float* h;                 // [R, I] fp32 (FP8) -- or null
+  uint16_t* hq_bf16;        // [R, I] bf16 (bf16 format) -- or null
+  float* amax_part;
+  WsHeader* hdr;
+  int R, I, E;
+  int fp8;
+};
+cudaError_t launch_finalize1(const Finalize1Args& a, int num_sms, cudaStream_t s);
+
+struct QuantHArgs {
+  const float* h;           // [R, I]
+  uint8_t* hq;              // [R, I] e4m3
+  const float* amax_part;
+  WsHeader* hdr;
+  int R, I;
+  float a2_static;
+};
+cudaError_t launch_quant_h(const QuantHArgs& a, int num_sms, cudaStream_t s);
+
+struct Finalize2Args {
+  const float* part;        // [S][R][H]
+  const int32_t* offsets;
+  const float* w2_scale;
+  const float* topk_w;      // [R] flattened
+  const int32_t* sorted_rows;
+  const WsHeader* hdr;
+  int32_t* status;
+  float* y;                 // [R, H]
+  int R, H, E;
+  int fp8;
+};
+cudaError_t launch_finalize2(const Finalize2Args& a, int num_sms, cudaStream_t s);
+
+struct CombineArgs {
+  const float* y;           // [R, H]
+  const int32_t* inv_perm;  // [R]
+  uint16_t* out;            // [T, H] bf16
+  int T, H, k;
+};
+cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+
+}  // namespace fmoe

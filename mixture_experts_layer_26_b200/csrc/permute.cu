@@ -1,0 +1,270 @@
+// Data shuffling: group the routed (token, slot) rows by expert, quantise the
+// activations while gathering them, and plan the grouped-GEMM work on the device.
+//
+// A fused MoE merges token routing, data shuffling and the expert networks into one
+// GPU operation (readmex.ai story "AWS details fused MoE kernel optimizations on
+// SageMaker", opening section).  The shuffle is the irregular, data-dependent part
+// (explore.n1n.ai "Mixture-of-Experts Kernel Engineering on Amazon SageMaker AI",
+// "The Core Bottlenecks of MoE Inference on H200 GPUs": irregular memory access and
+// dynamic per-expert batch sizes), so it is done here without any host round trip.
+//
+// permute_kernel (one CTA): per-expert histogram, exclusive scan into offsets, and a
+//   stable rank: row p of expert e lists the flattened indices t*k+j routed to e in
+//   ascending order (sorted_rows), inv_perm is its inverse.  It also turns the
+//   router's per-CTA max |x| into the per-tensor activation scale s1 = amax/448 and its
+//   inverse 448/amax (each one fp32 division; amax == 0 gives 1; a static scale s
+//   gives s and 1/s).
+// gather_kernel: A[p] = x[sorted_rows[p] / k], read with 16-byte loads and, for the
+//   FP8 format, multiplied by the inverse scale in fp32 and rounded to e4m3
+//   (round to nearest even, saturating at +-448).
+// plan_kernel (one warp): splits every expert's rows into chunks of at most
+//   chunk_rows rows and picks split-K factors for the swap-AB contractions.
+#include <cuda_fp8.h>
+
+#include "fmoe_kernels.h"
+
+namespace fmoe {
+
+namespace {
+
+constexpr int kPermThreads = 1024;
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int base[kMaxExperts];
+  __shared__ int ctot[kMaxExperts];
+  __shared__ int wc[kPermThreads / 32][kMaxExperts];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = a.E, R = a.R;
+
+  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < R; i += kPermThreads) {
+    const int e = a.topk_ids[i];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else record_status(&a.hdr->status, ST_BOUNDS);
+  }
+  __syncthreads();
+
+  // exclusive scan of the counts: lane l owns experts 8l .. 8l+7
+  if (warp == 0) {
+    int v[8], s = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      v[j] = e < E ? cnt[e] : 0;
+      s += v[j];
+    }
+    int incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    int run = incl - s;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) {
+        a.counts[e] = v[j];
+        a.offsets[e] = run;
+        base[e] = run;
+      }
+      run += v[j];
+    }
+    if (lane == 31) a.offsets[E] = incl;
+  }
+  if (tid == 32) {
+    // activation scale from the router's per-CTA maxima
+    float amax = 0.f;
+    const int n = a.hdr->router_ctas;
+    for (int i = 0; i < n; ++i) amax = fmaxf(amax, a.amax_part[i]);
+    float s1 = 1.f, inv1 = 1.f;
+    if (a.fp8) {
+      if (a.a1_static > 0.f) {
+        s1 = a.a1_static;
+        inv1 = 1.0f / a.a1_static;
+      } else if (amax > 0.f) {
+        s1 = amax / 448.0f;
+        inv1 = 448.0f / amax;
+      }
+    }
+    a.hdr->amax_x = amax;
+    a.hdr->s1 = s1;
+    a.hdr->inv1 = inv1;
+  }
+  __syncthreads();
+
+  // stable ranks, kPermThreads entries at a time
+  for (int c0 = 0; c0 < R; c0 += kPermThreads) {
+    for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) wc[i / E][i % E] = 0;
+    __syncthreads();
+    const int i = c0 + tid;
+    int e = i < R ? a.topk_ids[i] : E;
+    const bool valid = e >= 0 && e < E;
+    if (!valid) e = E;  // sentinel: matches only other invalid lanes
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && lane == __ffs(peers) - 1) wc[warp][e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += kPermThreads) {
+      int run = 0;
+      for (int w = 0; w < kPermThreads / 32; ++w) {
+        const int v = wc[w][ee];
+        wc[w][ee] = run;
+        run += v;
+      }
+      ctot[ee] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int pos = base[e] + wc[warp][e] + rank;
+      a.sorted_rows[pos] = i;
+      a.inv_perm[i] = pos;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += kPermThreads) base[ee] += ctot[ee];
+    __syncthreads();
+  }
+}
+
+constexpr int kGatherThreads = 256;
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// 8 bf16 (one uint4) times inv -> 8 e4m3 bytes (uint2)
+__device__ __forceinline__ uint2 quant8(const uint4& v, float inv) {
+  const float f0 = __uint_as_float(v.x << 16) * inv, f1 = __uint_as_float(v.x & 0xFFFF0000u) * inv;
+  const float f2 = __uint_as_float(v.y << 16) * inv, f3 = __uint_as_float(v.y & 0xFFFF0000u) * inv;
+  const float f4 = __uint_as_float(v.z << 16) * inv, f5 = __uint_as_float(v.z & 0xFFFF0000u) * inv;
+  const float f6 = __uint_as_float(v.w << 16) * inv, f7 = __uint_as_float(v.w & 0xFFFF0000u) * inv;
+  return make_uint2(e4m3x4(f0, f1, f2, f3), e4m3x4(f4, f5, f6, f7));
+}
+
+__global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * kGatherThreads) >> 5;
+  const float inv = a.fp8 ? a.hdr->inv1 : 1.f;
+  const int nvec = a.H / 16;  // 16 elements per step
+  for (int p = gwarp; p < a.R; p += nwarps) {
+    const int r = a.sorted_rows[p];
+    if (r < 0 || r >= a.R) {
+      if (lane == 0) record_status(a.status, ST_BOUNDS);
+      continue;
+    }
+    const int t = r / a.k;
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
+    if (a.fp8) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);
+      for (int v = lane; v < nvec; v += 32) {
+        const uint4 x0 = __ldg(src + 2 * v), x1 = __ldg(src + 2 * v + 1);
+        const uint2 q0 = quant8(x0, inv), q1 = quant8(x1, inv);
+        dst[v] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+      }
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);
+      for (int v = lane; v < 2 * nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+  }
+}
+
+// Split-K factor for `units` output tiles of `kblocks` K blocks on `sms` persistent
+// CTAs: the smallest factor whose last wave is at least 90% full, else the best one.
+__device__ int choose_split(int units, int kblocks, int smax, int sms) {
+  if (units <= 0) return 1;
+  const int cap = max(1, min(smax, kblocks / 2));
+  int best = 1;
+  float best_eff = -1.f;
+  for (int s = 1; s <= cap; ++s) {
+    const long u = static_cast<long>(units) * s;
+    const long waves = (u + sms - 1) / sms;
+    const float eff = static_cast<float>(u) / static_cast<float>(waves * sms);
+    if (eff >= 0.9f) return s;
+    if (eff > best_eff + 1e-6f) { best_eff = eff; best = s; }
+  }
+  return best;
+}
+
+__global__ void plan_kernel(PlanArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int CH = a.chunk_rows;
+  int n[8], nch[8], s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    n[j] = 0;
+    if (e < a.E) {
+      const int lo = a.offsets[e], hi = a.offsets[e + 1];
+      if (lo < 0 || hi < lo || hi > a.R) record_status(&a.hdr->status, ST_BOUNDS);
+      else n[j] = hi - lo;
+    }
+    nch[j] = (n[j] + CH - 1) / CH;
+    s += nch[j];
+  }
+  int incl = s;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int cb = incl - s;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    for (int c = 0; c < nch[j]; ++c) {
+      const int idx = cb + c;
+      if (idx >= a.max_chunks) {
+        record_status(&a.hdr->status, ST_BOUNDS);
+        break;
+      }
+      Chunk ch;
+      ch.e = e;
+      ch.row0 = a.offsets[e] + c * CH;
+      ch.nrows = min(CH, n[j] - c * CH);
+      ch.cb = cb;
+      ch.nch = nch[j];
+      ch.pad[0] = ch.pad[1] = ch.pad[2] = 0;
+      a.chunks[idx] = ch;
+    }
+    cb += nch[j];
+  }
+  if (lane == 0) {
+    const int nc = min(total, a.max_chunks);
+    a.hdr->n_chunks = nc;
+    if (a.swap_ab) {
+      a.hdr->split1 = choose_split(nc * a.units1_per_chunk, a.kblocks1, a.s1max, a.num_sms);
+      a.hdr->split2 = choose_split(nc * a.units2_per_chunk, a.kblocks2, a.s2max, a.num_sms);
+    } else {
+      a.hdr->split1 = 1;
+      a.hdr->split2 = 1;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
+  permute_kernel<<<1, kPermThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
+  const int rows_per_block = kGatherThreads / 32;
+  int grid = (a.R + rows_per_block - 1) / rows_per_block;
+  grid = grid < 1 ? 1 : grid;
+  gather_kernel<<<grid, kGatherThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
+  plan_kernel<<<1, 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fmoe

@@ -1,0 +1,149 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the header
+declares, sizes workspaces, and rejects bad arguments with the documented status
+codes before making any CUDA call (these tests run on machines without a GPU)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fused_moe.h")
+
+capi = pytest.importorskip("mixture_experts_layer_26_b200.capi",
+                           reason="libfused_moe.so not built")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FMOE_API\s+[\w\s\*]+?\b(fused_moe\w*)\s*\(", text)))
+
+
+def test_header_symbols_are_exported():
+    syms = header_symbols()
+    assert len(syms) == 14
+    assert set(syms) == set(capi.EXPORTED)
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_abi_version_and_strings():
+    assert capi.abi_version() == 1
+    for code, name in [(0, "FMOE_OK"), (1, "FMOE_ERR_INVALID_ARG"), (2, "FMOE_ERR_UNSUPPORTED"),
+                       (3, "FMOE_ERR_WORKSPACE"), (4, "FMOE_ERR_CUDA"), (5, "FMOE_ERR_TIMEOUT"),
+                       (6, "FMOE_ERR_DEVICE_BOUNDS")]:
+        assert capi.status_string(code) == name
+
+
+def dims(T=4, H=256, I=512, E=8, k=2, fp8=True, variant="auto"):
+    return capi.make_dims(T, H, I, E, k, fp8, variant)
+
+
+def test_workspace_size_valid_and_invalid():
+    assert capi.workspace_size(dims()) > 0
+    assert capi.workspace_size(dims(k=9)) == 0          # k > E
+    assert capi.workspace_size(dims(H=128)) == 0        # H % 256
+    assert capi.workspace_size(dims(I=100)) == 0        # I % 128
+    assert capi.workspace_size(dims(E=257, k=2)) == 0   # E > 256
+    assert capi.workspace_size(dims(T=-1)) == 0
+    # bigger problems need more workspace; the normal variant needs no split partials
+    assert capi.workspace_size(dims(T=64)) > capi.workspace_size(dims(T=4))
+    big_sw = capi.workspace_size(dims(T=64, H=4096, I=14336, variant="swap_ab"))
+    big_nm = capi.workspace_size(dims(T=64, H=4096, I=14336, variant="normal"))
+    assert big_sw > big_nm
+    # full-size workloads fit comfortably in HBM
+    assert capi.workspace_size(dims(T=4096, H=4096, I=14336)) < (2 << 30)
+    assert capi.workspace_size(dims(T=256, H=7168, I=2048, E=256, k=8)) < (1 << 30)
+
+
+FAKE = 1 << 20   # 16-byte aligned fake device addresses; never dereferenced
+
+
+class _T:
+    """Stands in for a tensor: data_ptr() and numel() only."""
+
+    def __init__(self, ptr, n=0):
+        self.p, self.n = ptr, n
+
+    def data_ptr(self):
+        return self.p
+
+    def numel(self):
+        return self.n
+
+
+def call_fused(d, x=FAKE, rw=FAKE, w13=FAKE, w2=FAKE, out=FAKE, ws=FAKE * 16, ws_bytes=None,
+               scales=True):
+    sc = capi.FmoeScales(FAKE, FAKE, 0.0, 0.0) if scales else None
+    if ws_bytes is None:
+        ws_bytes = capi.workspace_size(d) - 1           # always too small: no launch happens
+    return capi.fused_moe(d, _T(x), _T(rw), _T(w13), _T(w2), sc, _T(out), _T(ws, ws_bytes),
+                          stream=0, check=False)
+
+
+def test_validation_codes_without_cuda():
+    assert call_fused(dims(k=9)) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(k=0)) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(E=300)) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(T=-3)) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(H=384)) == capi.FMOE_ERR_UNSUPPORTED
+    assert call_fused(dims(I=64)) == capi.FMOE_ERR_UNSUPPORTED
+    assert call_fused(dims(H=16384 + 256)) == capi.FMOE_ERR_UNSUPPORTED
+    bad_variant = dims()
+    bad_variant.variant = 7
+    assert call_fused(bad_variant) == capi.FMOE_ERR_INVALID_ARG
+    bad_fmt = dims()
+    bad_fmt.wdtype = 3
+    assert call_fused(bad_fmt) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(), x=0) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(), out=0) == capi.FMOE_ERR_INVALID_ARG
+    assert call_fused(dims(), x=FAKE + 8) == capi.FMOE_ERR_UNSUPPORTED      # not 16-byte aligned
+    assert call_fused(dims(), scales=False) == capi.FMOE_ERR_INVALID_ARG   # FP8 needs scales
+    assert call_fused(dims()) == capi.FMOE_ERR_WORKSPACE                   # one byte short
+    assert call_fused(dims(), ws=FAKE * 16 + 128,
+                      ws_bytes=1 << 40) == capi.FMOE_ERR_WORKSPACE          # ws not 256-aligned
+    assert call_fused(dims(), ws=0, ws_bytes=1 << 40) == capi.FMOE_ERR_INVALID_ARG
+    # bf16 weights need no scales; still stops at the workspace check
+    assert call_fused(dims(fp8=False), scales=False) == capi.FMOE_ERR_WORKSPACE
+
+
+def test_launch_counts():
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="swap_ab")) == 10
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal")) == 8
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="swap_ab")) == 9
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="normal")) == 7
+    assert capi.fused_moe_launches_per_call(dims(T=0)) == 0
+    assert capi.fused_moe_launches_per_call(dims(k=9)) == -1
+    # AUTO: swap-AB while an expert averages at most 64 rows
+    assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 10
+    assert capi.fused_moe_launches_per_call(dims(T=257, E=8, k=2)) == 8
+
+
+def test_zero_tokens_is_a_noop():
+    # T == 0 returns OK after the dims checks, even with null buffers, and launches nothing
+    d = dims(T=0)
+    assert capi.fused_moe(d, _T(0), _T(0), _T(0), _T(0), None, _T(0), _T(0, 0), stream=0,
+                          check=False) == capi.FMOE_OK
+    assert capi.fused_moe_route(d, _T(0), _T(0), _T(0), _T(0), _T(0, 0), stream=0,
+                                check=False) == capi.FMOE_OK
+    assert capi.fused_moe_combine(d, _T(0), _T(0), _T(0), stream=0, check=False) == capi.FMOE_OK
+
+
+def test_step_validation():
+    d = dims()
+    small = _T(FAKE * 16, 10)
+    assert capi.fused_moe_route(d, _T(FAKE), _T(0), _T(FAKE), _T(FAKE), small, stream=0,
+                                check=False) == capi.FMOE_ERR_INVALID_ARG
+    assert capi.fused_moe_route(d, _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE), small, stream=0,
+                                check=False) == capi.FMOE_ERR_WORKSPACE
+    assert capi.fused_moe_permute(d, _T(FAKE), _T(FAKE), None, _T(FAKE), _T(FAKE), _T(FAKE),
+                                  _T(FAKE + 4), _T(FAKE), small, stream=0,
+                                  check=False) == capi.FMOE_ERR_UNSUPPORTED
+    assert capi.fused_moe_experts(d, _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE),
+                                  None, _T(FAKE), small, stream=0,
+                                  check=False) == capi.FMOE_ERR_INVALID_ARG    # FP8, no scales
+    assert capi.fused_moe_combine(d, _T(FAKE), _T(0), _T(FAKE), stream=0,
+                                  check=False) == capi.FMOE_ERR_INVALID_ARG
