@@ -207,6 +207,33 @@ FMOE_API fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, con
                                        float* ms_host, const char** names_host, int32_t cap,
                                        int32_t* n_host);
 
+/* Size of the library-owned workspace used by fused_moe_static_workspace: 64 MiB. */
+#define FUSED_MOE_STATIC_WS_BYTES ((size_t)64 << 20)
+
+/* fused_moe for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call; it exists for callers such as a plugin inside a serving
+ * process whose framework owns the GPU's memory pool and gives the plugin no
+ * allocator, or code that must not call cudaMalloc/cudaFree because they can
+ * synchronise the device.  It takes the same inputs and output as fused_moe but no
+ * workspace: the workspace is a file-scope device array of FUSED_MOE_STATIC_WS_BYTES
+ * that the library owns, and every GPU that loads the library holds it until the
+ * process exits.  It allocates nothing.
+ *   - Dims whose fused_moe_workspace_size exceeds FUSED_MOE_STATIC_WS_BYTES are
+ *     rejected with FMOE_ERR_WORKSPACE (use fused_moe with your own workspace).
+ *   - The first call on each device, with that device current, looks up the array's
+ *     device address; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; each call
+ *     clears the workspace header (device status word) first.  Calls that overlap on
+ *     the GPU race on the array: the caller must serialise them.
+ *   - device_status (device pointer to one int32, 4-byte aligned, may be NULL)
+ *     receives this call's device status word (FMOE_OK, FMOE_ERR_TIMEOUT or
+ *     FMOE_ERR_DEVICE_BOUNDS) when the stream reaches the end of the call. */
+FMOE_API fmoe_status fused_moe_static_workspace(const fmoe_dims* dims, const void* x,
+                                                const void* router_w, const void* w13,
+                                                const void* w2, const fmoe_scales* scales,
+                                                void* out, int32_t* device_status,
+                                                fmoe_stream stream);
+
 /* Synchronous: waits for `stream`, then returns the sticky device status recorded in
  * ws (FMOE_OK, FMOE_ERR_TIMEOUT or FMOE_ERR_DEVICE_BOUNDS), or FMOE_ERR_CUDA if the
  * wait or copy failed. */

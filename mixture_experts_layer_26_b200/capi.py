@@ -36,7 +36,9 @@ EXPORTED = (
     "fused_moe_workspace_init", "fused_moe_route", "fused_moe_permute", "fused_moe_experts",
     "fused_moe_combine", "fused_moe", "fused_moe_host_io", "fused_moe_get_device_status",
     "fused_moe_debug_scalars", "fused_moe_launches_per_call", "fused_moe_profile",
+    "fused_moe_static_workspace",
 )
+STATIC_WS_BYTES = 64 << 20  # FUSED_MOE_STATIC_WS_BYTES
 
 
 class FmoeDims(ctypes.Structure):
@@ -77,6 +79,8 @@ _dev_status = _sig("fused_moe_get_device_status", c_int32, c_void_p, c_void_p)
 _dbg = _sig("fused_moe_debug_scalars", c_int32, c_void_p, POINTER(c_float), POINTER(c_int32),
             c_void_p)
 _launches = _sig("fused_moe_launches_per_call", c_int32, _DP)
+_static_ws = _sig("fused_moe_static_workspace", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p,
+                  _SP, c_void_p, c_void_p, c_void_p)
 _profile = _sig("fused_moe_profile", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
                 c_void_p, c_void_p, c_size_t, c_void_p, POINTER(c_float), POINTER(c_char_p),
                 c_int32, POINTER(c_int32))
@@ -202,6 +206,15 @@ def fused_moe_debug_scalars(ws, stream=None):
     names_f = ("amax_x", "s1", "inv1", "amax_h", "s2", "inv2")
     names_i = ("n_chunks", "split1", "split2")
     return dict(zip(names_f, list(f))), dict(zip(names_i, list(i)))
+
+
+def fused_moe_static_workspace(dims, x, router_w, w13, w2, scales, out, device_status=None,
+                               stream=None, check=True) -> int:
+    """fused_moe without a caller workspace (library-owned 64 MiB device array)."""
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _static_ws(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(w13), _ptr(w2), sp,
+                    _ptr(out), _ptr(device_status), _stream(stream))
+    return _check(st, "fused_moe_static_workspace") if check else st
 
 
 def fused_moe_launches_per_call(dims) -> int:

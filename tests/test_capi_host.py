@@ -23,7 +23,7 @@ def header_symbols():
 
 def test_header_symbols_are_exported():
     syms = header_symbols()
-    assert len(syms) == 14
+    assert len(syms) == 15
     assert set(syms) == set(capi.EXPORTED)
     lib = ctypes.CDLL(capi.LIB_PATH)
     for s in syms:
