@@ -192,8 +192,8 @@ FMOE_API fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host
                               const void* w13, const void* w2, const fmoe_scales* scales,
                               void* out_host, void* ws, size_t ws_bytes, fmoe_stream stream);
 
-/* Number of kernels one fused_moe call launches for these dims (FP8: 8 NORMAL, 10
- * SWAP_AB; bf16: 7 NORMAL, 9 SWAP_AB; 0 for T == 0; -1 for invalid dims).  Host-only. */
+/* Number of kernels one fused_moe call launches for these dims (FP8: 7 NORMAL, 8
+ * SWAP_AB; bf16: 6 NORMAL, 7 SWAP_AB; 0 for T == 0; -1 for invalid dims).  Host-only. */
 FMOE_API int32_t fused_moe_launches_per_call(const fmoe_dims* dims);
 
 /* Measurement: runs fused_moe once with a CUDA event recorded on `stream` before the

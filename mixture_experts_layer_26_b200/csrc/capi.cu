@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -178,6 +179,20 @@ inline fmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FMOE_O
     if (_s != FMOE_OK) return _s;        \
   } while (0)
 
+}  // namespace
+
+namespace fmoe {
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("FMOE_DISABLE_PDL");
+    return !(v != nullptr && v[0] == '1');
+  }();
+  return on;
+}
+}  // namespace fmoe
+
+namespace {
+
 // Measurement hook: when active (fused_moe_profile only), every kernel launch of the
 // call sequence is followed by an event record on the launching stream.
 struct StageRecorder {
@@ -206,6 +221,23 @@ inline cudaError_t mark(const char* name, cudaStream_t s) {
 
 // ------------------------------------------------------------------ step bodies
 
+PlanParams plan_params(const fmoe_dims& d, const Layout& L, char* W) {
+  const int bk = L.fp8 ? 128 : 64;
+  PlanParams p{};
+  p.chunks = reinterpret_cast<Chunk*>(W + L.chunks);
+  p.chunk_rows = L.chunk_rows;
+  p.max_chunks = L.max_chunks;
+  p.swap_ab = L.swap ? 1 : 0;
+  p.units1_per_chunk = L.swap ? 2 * d.I / 128 : d.I / 128;
+  p.units2_per_chunk = L.swap ? d.H / 128 : d.H / 256;
+  p.kblocks1 = d.H / bk;
+  p.kblocks2 = d.I / bk;
+  p.s1max = std::max(L.s1max, 1);
+  p.s2max = std::max(L.s2max, 1);
+  p.num_sms = num_sms();
+  return p;
+}
+
 fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
                        int32_t* ids, float* tw, char* W, cudaStream_t s) {
   RouterArgs a{};
@@ -226,7 +258,7 @@ fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const
 
 fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids, const void* x,
                          const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
-                         int32_t* inv, void* a_perm, char* W, cudaStream_t s) {
+                         int32_t* inv, void* a_perm, char* W, cudaStream_t s, bool with_plan) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   PermuteArgs p{};
   p.topk_ids = ids;
@@ -241,7 +273,9 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   p.k = d.top_k;
   p.fp8 = L.fp8 ? 1 : 0;
   p.a1_static = sc != nullptr ? sc->a1_scale : 0.f;
-  FMOE_LAUNCH("permute", launch_permute(p, s), s);
+  p.with_plan = with_plan ? 1 : 0;
+  p.plan = plan_params(d, L, W);
+  FMOE_LAUNCH(with_plan ? "permute_plan" : "permute", launch_permute(p, s), s);
   GatherArgs g{};
   g.x = static_cast<const uint16_t*>(x);
   g.sorted_rows = rows;
@@ -256,10 +290,15 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   return FMOE_OK;
 }
 
+// Steps a3-a4.  plan_done: the permute launch already wrote the GEMM plan.  fused_out
+// (one-call path): in the swap-AB variant finish the second contraction's partials
+// straight into the combined output (needs ids and inv) instead of writing y.
 fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm,
                          const int32_t* offsets, const int32_t* rows, const float* tw,
                          const void* w13, const void* w2, const fmoe_scales* sc, float* y,
-                         char* W, cudaStream_t s) {
+                         char* W, cudaStream_t s, bool plan_done = false,
+                         void* fused_out = nullptr, const int32_t* ids = nullptr,
+                         const int32_t* inv = nullptr) {
   const int sms = num_sms();
   const bool fp8 = L.fp8, swap = L.swap;
   const int H = d.H, I = d.I, E = d.E, R = L.R;
@@ -270,23 +309,15 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   float* hbuf = reinterpret_cast<float*>(W + L.h);
   void* hq = W + L.hq;
 
-  PlanArgs pa{};
-  pa.offsets = offsets;
-  pa.chunks = chunks;
-  pa.hdr = hdr;
-  pa.R = R;
-  pa.E = E;
-  pa.chunk_rows = L.chunk_rows;
-  pa.max_chunks = L.max_chunks;
-  pa.swap_ab = swap ? 1 : 0;
-  pa.units1_per_chunk = swap ? 2 * I / 128 : I / 128;
-  pa.units2_per_chunk = swap ? H / 128 : H / 256;
-  pa.kblocks1 = H / bk;
-  pa.kblocks2 = I / bk;
-  pa.s1max = std::max(L.s1max, 1);
-  pa.s2max = std::max(L.s2max, 1);
-  pa.num_sms = sms;
-  FMOE_LAUNCH("plan", launch_plan(pa, s), s);
+  if (!plan_done) {
+    PlanArgs pa{};
+    pa.offsets = offsets;
+    pa.hdr = hdr;
+    pa.R = R;
+    pa.E = E;
+    pa.plan = plan_params(d, L, W);
+    FMOE_LAUNCH("plan", launch_plan(pa, s), s);
+  }
 
   const uint32_t xbox = swap ? 16u : 128u;
   GemmArgs g{};
@@ -353,7 +384,22 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g2.rows_per_expert = H;
   FMOE_LAUNCH(swap ? "gemm2_swapab" : "gemm2_normal", launch_gemm(g2, fp8, swap, 2, sms, s), s);
 
-  if (swap) {
+  if (swap && fused_out != nullptr) {
+    CombinePartialsArgs c{};
+    c.part = reinterpret_cast<const float*>(W + L.p2);
+    c.inv_perm = inv;
+    c.topk_ids = ids;
+    c.topk_w = tw;
+    c.w2_scale = fp8 ? sc->w2_scale : nullptr;
+    c.hdr = hdr;
+    c.out = static_cast<uint16_t*>(fused_out);
+    c.T = d.T;
+    c.H = H;
+    c.k = d.top_k;
+    c.E = E;
+    c.fp8 = fp8 ? 1 : 0;
+    FMOE_LAUNCH("combine_partials", launch_combine_partials(c, sms, s), s);
+  } else if (swap) {
     Finalize2Args f{};
     f.part = reinterpret_cast<const float*>(W + L.p2);
     f.offsets = offsets;
@@ -396,8 +442,11 @@ fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   int32_t* inv = reinterpret_cast<int32_t*>(W + L.inv);
   float* y = reinterpret_cast<float*>(W + L.y);
   FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
-  FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s));
-  FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s));
+  FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s,
+                        /*with_plan=*/true));
+  FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s,
+                        /*plan_done=*/true, /*fused_out=*/out, ids, inv));
+  if (L.swap) return FMOE_OK;  // combined by combine_partials
   return combine_impl(d, y, inv, out, s);
 }
 
@@ -455,7 +504,8 @@ fmoe_status fused_moe_permute(const fmoe_dims* dims, const int32_t* topk_ids, co
   const Layout L = make_layout(*dims);
   FMOE_TRY(check_ws(L, ws, ws_bytes));
   return permute_impl(*dims, L, topk_ids, x, scales, counts, offsets, sorted_rows, inv_perm,
-                      a_perm, static_cast<char*>(ws), static_cast<cudaStream_t>(stream));
+                      a_perm, static_cast<char*>(ws), static_cast<cudaStream_t>(stream),
+                      /*with_plan=*/false);
 }
 
 fmoe_status fused_moe_experts(const fmoe_dims* dims, const void* a_perm, const int32_t* offsets,
@@ -519,8 +569,8 @@ int32_t fused_moe_launches_per_call(const fmoe_dims* dims) {
   if (check_dims(dims) != FMOE_OK) return -1;
   if (dims->T == 0) return 0;
   const Layout L = make_layout(*dims);
-  // router, permute, gather, plan, gemm1, [finalize1], [quant_h], gemm2, [finalize2], combine
-  return 7 + (L.swap ? 2 : 0) + (L.fp8 ? 1 : 0);
+  // router, permute (+plan), gather, gemm1, [finalize1], [quant_h], gemm2, combine
+  return 6 + (L.swap ? 1 : 0) + (L.fp8 ? 1 : 0);
 }
 
 fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, const void* router_w,

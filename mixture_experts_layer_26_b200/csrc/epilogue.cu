@@ -50,6 +50,8 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 __global__ void __launch_bounds__(kEwThreads) finalize1_kernel(Finalize1Args a) {
   __shared__ int offs[kMaxExperts + 1];
   __shared__ float red[kEwThreads / 32];
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];
   __syncthreads();
   const int S = a.hdr->split1;
@@ -105,6 +107,8 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 
 __global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
   __shared__ float s_inv;
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x < 32) {
     float m = 0.f;
     const int n = a.hdr->amax_h_count;
@@ -146,6 +150,8 @@ __global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
 
 __global__ void __launch_bounds__(kEwThreads) finalize2_kernel(Finalize2Args a) {
   __shared__ int offs[kMaxExperts + 1];
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];
   __syncthreads();
   const int S = a.hdr->split2;
@@ -178,7 +184,59 @@ __global__ void __launch_bounds__(kEwThreads) finalize2_kernel(Finalize2Args a) 
   }
 }
 
+__device__ __forceinline__ uint4 pack_bf16x8(const float* acc) {
+  uint4 o;
+  __nv_bfloat162 b;
+  b = __floats2bfloat162_rn(acc[0], acc[1]); o.x = *reinterpret_cast<uint32_t*>(&b);
+  b = __floats2bfloat162_rn(acc[2], acc[3]); o.y = *reinterpret_cast<uint32_t*>(&b);
+  b = __floats2bfloat162_rn(acc[4], acc[5]); o.z = *reinterpret_cast<uint32_t*>(&b);
+  b = __floats2bfloat162_rn(acc[6], acc[7]); o.w = *reinterpret_cast<uint32_t*>(&b);
+  return o;
+}
+
+// Same arithmetic, in the same order, as finalize2 followed by combine.
+__global__ void __launch_bounds__(kEwThreads) combine_partials_kernel(CombinePartialsArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int S = a.hdr->split2;
+  const float s2 = a.fp8 ? a.hdr->s2 : 1.f;
+  const int H8 = a.H / 8;
+  const int R = a.T * a.k;
+  const size_t plane = static_cast<size_t>(R) * a.H;
+  const size_t total = static_cast<size_t>(a.T) * H8;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const int t = static_cast<int>(idx / H8), c = static_cast<int>(idx % H8) * 8;
+    float acc[8];
+    for (int j = 0; j < a.k; ++j) {
+      const size_t q = static_cast<size_t>(t) * a.k + j;
+      int p = a.inv_perm[q];
+      int e = a.topk_ids[q];
+      if (p < 0 || p >= R) p = 0;  // malformed inputs: stay in bounds
+      if (e < 0 || e >= a.E) e = 0;
+      const float sc = a.fp8 ? s2 * a.w2_scale[e] : 1.f;
+      const float wr = a.topk_w[q];
+      const float* src = a.part + static_cast<size_t>(p) * a.H + c;
+      float4 v0 = *reinterpret_cast<const float4*>(src);
+      float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+      for (int s = 1; s < S; ++s) {
+        const float4 u0 = *reinterpret_cast<const float4*>(src + s * plane);
+        const float4 u1 = *reinterpret_cast<const float4*>(src + s * plane + 4);
+        v0.x += u0.x; v0.y += u0.y; v0.z += u0.z; v0.w += u0.w;
+        v1.x += u1.x; v1.y += u1.y; v1.z += u1.z; v1.w += u1.w;
+      }
+      const float y[8] = {v0.x * sc * wr, v0.y * sc * wr, v0.z * sc * wr, v0.w * sc * wr,
+                          v1.x * sc * wr, v1.y * sc * wr, v1.z * sc * wr, v1.w * sc * wr};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = (j == 0) ? y[i] : acc[i] + y[i];
+    }
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = pack_bf16x8(acc);
+  }
+}
+
 __global__ void __launch_bounds__(kEwThreads) combine_kernel(CombineArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int H8 = a.H / 8;
   const size_t total = static_cast<size_t>(a.T) * H8;
   for (size_t idx = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; idx < total;
@@ -198,13 +256,7 @@ __global__ void __launch_bounds__(kEwThreads) combine_kernel(CombineArgs a) {
         acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
       }
     }
-    uint4 o;
-    __nv_bfloat162 b;
-    b = __floats2bfloat162_rn(acc[0], acc[1]); o.x = *reinterpret_cast<uint32_t*>(&b);
-    b = __floats2bfloat162_rn(acc[2], acc[3]); o.y = *reinterpret_cast<uint32_t*>(&b);
-    b = __floats2bfloat162_rn(acc[4], acc[5]); o.z = *reinterpret_cast<uint32_t*>(&b);
-    b = __floats2bfloat162_rn(acc[6], acc[7]); o.w = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = o;
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = pack_bf16x8(acc);
   }
 }
 
@@ -222,23 +274,28 @@ int ew_grid(size_t work_items, int num_sms) {
 cudaError_t launch_finalize1(const Finalize1Args& a, int num_sms, cudaStream_t s) {
   int grid = ew_grid(static_cast<size_t>(a.R) * a.I / 4, num_sms);
   if (grid > kAmaxSlots) grid = kAmaxSlots;
-  finalize1_kernel<<<grid, kEwThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(finalize1_kernel, dim3(grid), dim3(kEwThreads), 0, s, a);
 }
 
 cudaError_t launch_quant_h(const QuantHArgs& a, int num_sms, cudaStream_t s) {
-  quant_h_kernel<<<ew_grid(static_cast<size_t>(a.R) * a.I / 16, num_sms), kEwThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(quant_h_kernel, dim3(ew_grid(static_cast<size_t>(a.R) * a.I / 16, num_sms)),
+                  dim3(kEwThreads), 0, s, a);
 }
 
 cudaError_t launch_finalize2(const Finalize2Args& a, int num_sms, cudaStream_t s) {
-  finalize2_kernel<<<ew_grid(static_cast<size_t>(a.R) * a.H / 4, num_sms), kEwThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(finalize2_kernel, dim3(ew_grid(static_cast<size_t>(a.R) * a.H / 4, num_sms)),
+                  dim3(kEwThreads), 0, s, a);
 }
 
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
-  combine_kernel<<<ew_grid(static_cast<size_t>(a.T) * a.H / 8, num_sms), kEwThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(combine_kernel, dim3(ew_grid(static_cast<size_t>(a.T) * a.H / 8, num_sms)),
+                  dim3(kEwThreads), 0, s, a);
+}
+
+cudaError_t launch_combine_partials(const CombinePartialsArgs& a, int num_sms, cudaStream_t s) {
+  return launch_k(combine_partials_kernel,
+                  dim3(ew_grid(static_cast<size_t>(a.T) * a.H / 8, num_sms)), dim3(kEwThreads), 0,
+                  s, a);
 }
 
 }  // namespace fmoe

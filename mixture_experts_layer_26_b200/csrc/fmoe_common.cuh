@@ -75,6 +75,21 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ------------------------------------------------------------------------------------
+// programmatic dependent launch
+//
+// Every kernel of the library is launched with programmatic stream serialisation, so
+// it may start while its predecessor in the stream is still running.  Each kernel
+// calls griddep_wait() before its first global-memory access that depends on earlier
+// work in the stream, and calls griddep_launch_dependents() only after that wait.
+// Hence when a kernel starts, the kernel two places before it has completed.
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

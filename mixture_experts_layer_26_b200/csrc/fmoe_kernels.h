@@ -24,6 +24,27 @@ inline cudaError_t set_max_dynamic_smem(int bytes) {
   return err;
 }
 
+// Launch with programmatic stream serialisation (see griddep_wait in fmoe_common.cuh).
+// FMOE_DISABLE_PDL=1 in the environment launches plainly instead (a debugging aid).
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // ----------------------------------------------------------------------------- router
 struct RouterArgs {
   const uint16_t* x;    // [T, H] bf16 bits
@@ -39,6 +60,18 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 int router_tokens_per_cta(int T, int H, int E, int num_sms);
 
 // ----------------------------------------------------------------------------- permute
+// How the grouped GEMMs are planned from the per-expert offsets.
+struct PlanParams {
+  Chunk* chunks;           // [max_chunks]
+  int chunk_rows, max_chunks;
+  int swap_ab;
+  int units1_per_chunk;    // output tiles of the first contraction per chunk
+  int units2_per_chunk;
+  int kblocks1, kblocks2;  // K blocks of each contraction
+  int s1max, s2max;        // largest split-K factors the workspace holds
+  int num_sms;
+};
+
 struct PermuteArgs {
   const int32_t* topk_ids;  // [R]
   int32_t* counts;          // [E]
@@ -50,6 +83,8 @@ struct PermuteArgs {
   int R, E, k;
   int fp8;                  // compute the activation scale (FP8 format)
   float a1_static;          // > 0: static scale
+  int with_plan;            // also write the GEMM plan (one-call path)
+  PlanParams plan;
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 
@@ -67,15 +102,9 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
 // ----------------------------------------------------------------------------- experts
 struct PlanArgs {
   const int32_t* offsets;  // [E + 1]
-  Chunk* chunks;           // [max_chunks]
   WsHeader* hdr;
-  int R, E, chunk_rows, max_chunks;
-  int swap_ab;
-  int units1_per_chunk;    // output tiles of the first contraction per chunk
-  int units2_per_chunk;
-  int kblocks1, kblocks2;  // K blocks of each contraction
-  int s1max, s2max;        // largest split-K factors the workspace holds
-  int num_sms;
+  int R, E;
+  PlanParams plan;
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 
@@ -139,6 +168,21 @@ struct Finalize2Args {
   int fp8;
 };
 cudaError_t launch_finalize2(const Finalize2Args& a, int num_sms, cudaStream_t s);
+
+// finalize2 and combine in one pass (one-call swap-AB path): out[t] = bf16(sum over j of
+// (sum over s of part[s][p_j]) * s2 * w2_scale[e_j] * topk_w[t*k+j]), p_j = inv_perm[t*k+j].
+struct CombinePartialsArgs {
+  const float* part;        // [S][R][H]
+  const int32_t* inv_perm;  // [R]
+  const int32_t* topk_ids;  // [R]
+  const float* topk_w;      // [R]
+  const float* w2_scale;    // [E] or null
+  const WsHeader* hdr;
+  uint16_t* out;            // [T, H] bf16
+  int T, H, k, E;
+  int fp8;
+};
+cudaError_t launch_combine_partials(const CombinePartialsArgs& a, int num_sms, cudaStream_t s);
 
 struct CombineArgs {
   const float* y;           // [R, H]

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   constexpr int kBK = kFp8 ? 128 : 64;  // K elements per stage (128 bytes per row)
   const int KB = a.K / kBK;
 
+  // Set-up that reads nothing produced earlier in the stream: barriers, TMEM, descriptors.
   if (threadIdx.x == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&ctl.full[s], 1);
@@ -117,8 +118,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     mbar_init(&ctl.drain, 1);
     ctl.abort_flag = 0;
     ctl.amax_bits = 0;
-    ctl.n_chunks = a.hdr->n_chunks;
-    ctl.split = kSwap ? (kGemm == 1 ? a.hdr->split1 : a.hdr->split2) : 1;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -130,9 +129,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // The first contraction's work list is written by the kernel right before it, so it
+  // waits here.  The second contraction's work list was written at least two kernels
+  // earlier, which has completed by the time this grid starts (every kernel triggers
+  // its dependents only after its own wait), so its weight tiles are prefetched before
+  // waiting for the activations.
+  constexpr bool kPrefetch = (kGemm == 2);
+  if constexpr (!kPrefetch) griddep_wait();
+  if (threadIdx.x == 0) {
+    ctl.n_chunks = a.hdr->n_chunks;
+    ctl.split = kSwap ? (kGemm == 1 ? a.hdr->split1 : a.hdr->split2) : 1;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (!kPrefetch) {
+    if (threadIdx.x == 0) griddep_launch_dependents();
+  }
 
   const uint32_t tmem_base = ctl.tmem_base;
   const int S = ctl.split > 0 ? ctl.split : 1;
@@ -151,39 +164,101 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (long u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        const Unit t = decode_unit(u, a.chunks, per_chunk, S, KB);
-        const int nbox = kSwap ? (t.nrows + kSwapBoxRows - 1) / kSwapBoxRows : 1;
-        const uint32_t bytes = kSwap ? kTileA + nbox * kSwapBoxRows * 128 : 3 * kTileA;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, a.status, budget)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + stage * stage_bytes;
-          uint8_t* sb = sa + kTileA;
-          mbar_arrive_expect_tx(&ctl.full[stage], bytes);
-          const int kx = kb * kBK;
-          if (kSwap) {
-            tma_load_2d(sa, &a.map_w, &ctl.full[stage], kx, t.e * a.rows_per_expert + t.tile * 128,
-                        pol_w);
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(sb + b * kSwapBoxRows * 128, &a.map_x, &ctl.full[stage], kx,
-                          t.row0 + b * kSwapBoxRows, pol_x);
-          } else {
-            tma_load_2d(sa, &a.map_x, &ctl.full[stage], kx, t.row0, pol_x);
-            const int wrow = t.e * a.rows_per_expert + (kGemm == 1 ? t.tile * 128 : t.tile * 256);
-            tma_load_2d(sb, &a.map_w, &ctl.full[stage], kx, wrow, pol_w);
-            tma_load_2d(sb + kTileA, &a.map_w, &ctl.full[stage], kx,
-                        kGemm == 1 ? wrow + a.I : wrow + 128, pol_w);
-          }
-          issued_mask |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == nst) {
-            stage = 0;
-            phase ^= 1u;
+
+      struct Cursor {
+        long u;
+        int kb;
+        bool have;
+        Unit t;
+      };
+      auto cursor_start = [&](Cursor& c) {
+        c.u = blockIdx.x;
+        c.have = c.u < total;
+        if (c.have) {
+          c.t = decode_unit(c.u, a.chunks, per_chunk, S, KB);
+          c.kb = c.t.kb0;
+        }
+      };
+      auto cursor_next = [&](Cursor& c) {
+        if (++c.kb >= c.t.kb1) {
+          c.u += gridDim.x;
+          c.have = c.u < total;
+          if (c.have) {
+            c.t = decode_unit(c.u, a.chunks, per_chunk, S, KB);
+            c.kb = c.t.kb0;
           }
         }
+      };
+      auto nbox_of = [&](const Unit& t) { return kSwap ? (t.nrows + kSwapBoxRows - 1) / kSwapBoxRows : 1; };
+      auto tx_bytes = [&](const Unit& t) -> uint32_t {
+        return kSwap ? kTileA + nbox_of(t) * kSwapBoxRows * 128 : 3 * kTileA;
+      };
+      // weight tile(s) of one stage
+      auto load_w = [&](int st, const Unit& t, int kb) {
+        uint8_t* sa = smem + st * stage_bytes;
+        const int kx = kb * kBK;
+        if (kSwap) {
+          tma_load_2d(sa, &a.map_w, &ctl.full[st], kx, t.e * a.rows_per_expert + t.tile * 128, pol_w);
+        } else {
+          uint8_t* sb = sa + kTileA;
+          const int wrow = t.e * a.rows_per_expert + (kGemm == 1 ? t.tile * 128 : t.tile * 256);
+          tma_load_2d(sb, &a.map_w, &ctl.full[st], kx, wrow, pol_w);
+          tma_load_2d(sb + kTileA, &a.map_w, &ctl.full[st], kx, kGemm == 1 ? wrow + a.I : wrow + 128,
+                      pol_w);
+        }
+      };
+      // activation tile(s) of one stage
+      auto load_x = [&](int st, const Unit& t, int kb) {
+        uint8_t* sa = smem + st * stage_bytes;
+        const int kx = kb * kBK;
+        if (kSwap) {
+          uint8_t* sb = sa + kTileA;
+          for (int b = 0; b < nbox_of(t); ++b)
+            tma_load_2d(sb + b * kSwapBoxRows * 128, &a.map_x, &ctl.full[st], kx,
+                        t.row0 + b * kSwapBoxRows, pol_x);
+        } else {
+          tma_load_2d(sa, &a.map_x, &ctl.full[st], kx, t.row0, pol_x);
+        }
+      };
+      auto bump = [&]() {
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == nst) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+
+      Cursor cur;
+      cursor_start(cur);
+      if constexpr (kPrefetch) {
+        // weights of the first stages (fresh stages: nothing to wait for)
+        Cursor first = cur;
+        int npre = 0;
+        while (cur.have && npre < nst) {
+          mbar_arrive_expect_tx(&ctl.full[stage], tx_bytes(cur.t));
+          load_w(stage, cur.t, cur.kb);
+          bump();
+          ++npre;
+          cursor_next(cur);
+        }
+        griddep_wait();
+        griddep_launch_dependents();
+        for (int i = 0; i < npre; ++i) {  // their activations, now that they are written
+          load_x(i, first.t, first.kb);
+          cursor_next(first);
+        }
+      }
+      while (cur.have) {
+        if (!mbar_wait(&ctl.empty[stage], phase ^ 1u, abort_flag, a.status, budget)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&ctl.full[stage], tx_bytes(cur.t));
+        load_w(stage, cur.t, cur.kb);
+        load_x(stage, cur.t, cur.kb);
+        bump();
+        cursor_next(cur);
       }
       if (!ok) {
         // aborted: let every copy this thread issued land before the CTA exits
@@ -193,6 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             mbar_wait(&ctl.full[s], (issued_parity >> s) & 1u, &dummy, a.status, budget);
           }
       }
+    } else if (kPrefetch) {
+      // lanes that do not produce still order their later reads after the wait
+      griddep_wait();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -244,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------- epilogue
+    if constexpr (kPrefetch) griddep_wait();  // scales and routing weights of this call
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
     int acc = 0;
@@ -359,8 +438,7 @@ cudaError_t launch_one(const GemmArgs& a, int num_sms, cudaStream_t s) {
   const size_t smem = 1024 + static_cast<size_t>(a.nstages) * stage_bytes;
   cudaError_t err = set_max_dynamic_smem<gemm_kernel<kFp8, kSwap, kGemm>>(kSmemBudget + 1024);
   if (err != cudaSuccess) return err;
-  gemm_kernel<kFp8, kSwap, kGemm><<<num_sms, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(gemm_kernel<kFp8, kSwap, kGemm>, dim3(num_sms), dim3(kThreads), smem, s, a);
 }
 
 }  // namespace

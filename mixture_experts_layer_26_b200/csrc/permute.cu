@@ -29,15 +29,95 @@ namespace {
 
 constexpr int kPermThreads = 1024;
 
+// Split-K factor for `units` output tiles of `kblocks` K blocks on `sms` persistent
+// CTAs: the smallest factor whose last wave is at least 90% full, else the best one.
+__device__ int choose_split(int units, int kblocks, int smax, int sms) {
+  if (units <= 0) return 1;
+  const int cap = max(1, min(smax, kblocks / 2));
+  int best = 1;
+  float best_eff = -1.f;
+  for (int s = 1; s <= cap; ++s) {
+    const long u = static_cast<long>(units) * s;
+    const long waves = (u + sms - 1) / sms;
+    const float eff = static_cast<float>(u) / static_cast<float>(waves * sms);
+    if (eff >= 0.9f) return s;
+    if (eff > best_eff + 1e-6f) { best_eff = eff; best = s; }
+  }
+  return best;
+}
+
+// One warp: split every expert's rows [offsets[e], offsets[e+1]) into chunks of at most
+// chunk_rows rows, write the chunk list and the split-K factors.  `offsets` may live in
+// shared or global memory; malformed offsets are reported and treated as empty.
+__device__ void build_plan(const int* offsets, int E, int R, const PlanParams& p, WsHeader* hdr) {
+  const int lane = threadIdx.x & 31;
+  const int CH = p.chunk_rows;
+  int n[8], nch[8], s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    n[j] = 0;
+    if (e < E) {
+      const int lo = offsets[e], hi = offsets[e + 1];
+      if (lo < 0 || hi < lo || hi > R) record_status(&hdr->status, ST_BOUNDS);
+      else n[j] = hi - lo;
+    }
+    nch[j] = (n[j] + CH - 1) / CH;
+    s += nch[j];
+  }
+  int incl = s;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int cb = incl - s;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    for (int c = 0; c < nch[j]; ++c) {
+      const int idx = cb + c;
+      if (idx >= p.max_chunks) {
+        record_status(&hdr->status, ST_BOUNDS);
+        break;
+      }
+      Chunk ch;
+      ch.e = e;
+      ch.row0 = offsets[e] + c * CH;
+      ch.nrows = min(CH, n[j] - c * CH);
+      ch.cb = cb;
+      ch.nch = nch[j];
+      ch.pad[0] = ch.pad[1] = ch.pad[2] = 0;
+      p.chunks[idx] = ch;
+    }
+    cb += nch[j];
+  }
+  if (lane == 0) {
+    const int nc = min(total, p.max_chunks);
+    hdr->n_chunks = nc;
+    if (p.swap_ab) {
+      hdr->split1 = choose_split(nc * p.units1_per_chunk, p.kblocks1, p.s1max, p.num_sms);
+      hdr->split2 = choose_split(nc * p.units2_per_chunk, p.kblocks2, p.s2max, p.num_sms);
+    } else {
+      hdr->split1 = 1;
+      hdr->split2 = 1;
+    }
+  }
+}
+
+
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
   __shared__ int cnt[kMaxExperts];
-  __shared__ int base[kMaxExperts];
+  __shared__ int base[kMaxExperts + 1];
   __shared__ int ctot[kMaxExperts];
   __shared__ int wc[kPermThreads / 32][kMaxExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, R = a.R;
 
   for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
   for (int i = tid; i < R; i += kPermThreads) {
     const int e = a.topk_ids[i];
@@ -72,7 +152,10 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
       }
       run += v[j];
     }
-    if (lane == 31) a.offsets[E] = incl;
+    if (lane == 31) {
+      a.offsets[E] = incl;
+      base[E] = incl;
+    }
   }
   if (tid == 32) {
     // activation scale from the router's per-CTA maxima
@@ -93,6 +176,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
     a.hdr->s1 = s1;
     a.hdr->inv1 = inv1;
   }
+  __syncthreads();
+  if (a.with_plan && warp == 0) build_plan(base, E, R, a.plan, a.hdr);
   __syncthreads();
 
   // stable ranks, kPermThreads entries at a time
@@ -149,6 +234,8 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
   const int lane = threadIdx.x & 31;
   const int gwarp = (blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * kGatherThreads) >> 5;
+  griddep_wait();
+  griddep_launch_dependents();
   const float inv = a.fp8 ? a.hdr->inv1 : 1.f;
   const int nvec = a.H / 16;  // 16 elements per step
   for (int p = gwarp; p < a.R; p += nwarps) {
@@ -173,98 +260,27 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
   }
 }
 
-// Split-K factor for `units` output tiles of `kblocks` K blocks on `sms` persistent
-// CTAs: the smallest factor whose last wave is at least 90% full, else the best one.
-__device__ int choose_split(int units, int kblocks, int smax, int sms) {
-  if (units <= 0) return 1;
-  const int cap = max(1, min(smax, kblocks / 2));
-  int best = 1;
-  float best_eff = -1.f;
-  for (int s = 1; s <= cap; ++s) {
-    const long u = static_cast<long>(units) * s;
-    const long waves = (u + sms - 1) / sms;
-    const float eff = static_cast<float>(u) / static_cast<float>(waves * sms);
-    if (eff >= 0.9f) return s;
-    if (eff > best_eff + 1e-6f) { best_eff = eff; best = s; }
-  }
-  return best;
-}
-
 __global__ void plan_kernel(PlanArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int CH = a.chunk_rows;
-  int n[8], nch[8], s = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane * 8 + j;
-    n[j] = 0;
-    if (e < a.E) {
-      const int lo = a.offsets[e], hi = a.offsets[e + 1];
-      if (lo < 0 || hi < lo || hi > a.R) record_status(&a.hdr->status, ST_BOUNDS);
-      else n[j] = hi - lo;
-    }
-    nch[j] = (n[j] + CH - 1) / CH;
-    s += nch[j];
-  }
-  int incl = s;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += t;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  int cb = incl - s;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane * 8 + j;
-    for (int c = 0; c < nch[j]; ++c) {
-      const int idx = cb + c;
-      if (idx >= a.max_chunks) {
-        record_status(&a.hdr->status, ST_BOUNDS);
-        break;
-      }
-      Chunk ch;
-      ch.e = e;
-      ch.row0 = a.offsets[e] + c * CH;
-      ch.nrows = min(CH, n[j] - c * CH);
-      ch.cb = cb;
-      ch.nch = nch[j];
-      ch.pad[0] = ch.pad[1] = ch.pad[2] = 0;
-      a.chunks[idx] = ch;
-    }
-    cb += nch[j];
-  }
-  if (lane == 0) {
-    const int nc = min(total, a.max_chunks);
-    a.hdr->n_chunks = nc;
-    if (a.swap_ab) {
-      a.hdr->split1 = choose_split(nc * a.units1_per_chunk, a.kblocks1, a.s1max, a.num_sms);
-      a.hdr->split2 = choose_split(nc * a.units2_per_chunk, a.kblocks2, a.s2max, a.num_sms);
-    } else {
-      a.hdr->split1 = 1;
-      a.hdr->split2 = 1;
-    }
-  }
+  griddep_wait();
+  griddep_launch_dependents();
+  build_plan(a.offsets, a.E, a.R, a.plan, a.hdr);
 }
 
 }  // namespace
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
-  permute_kernel<<<1, kPermThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(permute_kernel, dim3(1), dim3(kPermThreads), 0, s, a);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
   const int rows_per_block = kGatherThreads / 32;
   int grid = (a.R + rows_per_block - 1) / rows_per_block;
   grid = grid < 1 ? 1 : grid;
-  gather_kernel<<<grid, kGatherThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(gather_kernel, dim3(grid), dim3(kGatherThreads), 0, s, a);
 }
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
-  plan_kernel<<<1, 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(plan_kernel, dim3(1), dim3(32), 0, s, a);
 }
 
 }  // namespace fmoe

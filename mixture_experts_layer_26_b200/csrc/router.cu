@@ -57,6 +57,9 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   const int H = a.H, E = a.E;
   const int vec_per_row = H / 8;  // 16-byte vectors per row
 
+  griddep_wait();
+  griddep_launch_dependents();
+
   // ---- stage x rows (zero for tokens past T) and their max |x|
   float amax = 0.f;
   for (int i = threadIdx.x; i < TB * vec_per_row; i += kRouterThreads) {
@@ -169,8 +172,7 @@ cudaError_t launch_tb(const RouterArgs& a, cudaStream_t s) {
   cudaError_t err = set_max_dynamic_smem<router_kernel<TB, EG>>(160 * 1024);
   if (err != cudaSuccess) return err;
   const int grid = (a.T + TB - 1) / TB;
-  router_kernel<TB, EG><<<grid, kRouterThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(router_kernel<TB, EG>, dim3(grid), dim3(kRouterThreads), smem, s, a);
 }
 
 template <int TB>

@@ -111,15 +111,15 @@ def test_validation_codes_without_cuda():
 
 
 def test_launch_counts():
-    assert capi.fused_moe_launches_per_call(dims(T=4, variant="swap_ab")) == 10
-    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal")) == 8
-    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="swap_ab")) == 9
-    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="normal")) == 7
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="swap_ab")) == 8
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal")) == 7
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="swap_ab")) == 7
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="normal")) == 6
     assert capi.fused_moe_launches_per_call(dims(T=0)) == 0
     assert capi.fused_moe_launches_per_call(dims(k=9)) == -1
     # AUTO: swap-AB while an expert averages at most 64 rows
-    assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 10
-    assert capi.fused_moe_launches_per_call(dims(T=257, E=8, k=2)) == 8
+    assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 8
+    assert capi.fused_moe_launches_per_call(dims(T=257, E=8, k=2)) == 7
 
 
 def test_zero_tokens_is_a_noop():
