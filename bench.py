@@ -373,21 +373,37 @@ def run_ours(args, rank, world, local_rank):
     esz = 1 if fp8 else 2
     peaks, peak_kind = load_peaks()
     dom = max(kern_ms, key=kern_ms.get)
+    variant = "swap_ab" if "swapab" in "".join(kern_ms) else "normal"
     gemm1_bytes = touched * 2 * s.H * s.I * esz          # weights of the touched experts
     gemm2_bytes = touched * s.H * s.I * esz
-    algo = {"gemm1": gemm1_bytes, "gemm2": gemm2_bytes}
-    dom_bytes = algo.get(dom.split("_")[0])
-    variant = "swap_ab" if "swapab" in "".join(kern_ms) else "normal"
+    gemm1_flops = 4.0 * s.R * s.H * s.I                  # gate and up: 2 x (2 R H I)
+    gemm2_flops = 2.0 * s.R * s.H * s.I
+    kind = dom.split("_")[0]
     roof = None
-    if dom_bytes is not None:
+    traffic = profiled_traffic(dom, f"{args.workload}_T{s.T}")
+    if variant == "swap_ab" and kind in ("gemm1", "gemm2"):
+        dom_bytes = gemm1_bytes if kind == "gemm1" else gemm2_bytes
         ach = dom_bytes / (kern_ms[dom] / 1e3) / 1e9
-        traffic = profiled_traffic(dom, f"{args.workload}_T{s.T}")
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": dom, "kernel_us": round(1e3 * kern_ms[dom], 2),
                 "algorithmic_bytes": dom_bytes,
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"}
+    elif kind in ("gemm1", "gemm2"):
+        dom_flops = gemm1_flops if kind == "gemm1" else gemm2_flops
+        # a contraction timed inside a long back-to-back step: the sustained peak; FP8 is
+        # the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 = 2
+        ratio = 2.0 if fp8 else 1.0
+        peak = ratio * peaks["bf16_tflops_sustained"]
+        ach = dom_flops / (kern_ms[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
+                "kernel": dom, "kernel_us": round(1e3 * kern_ms[dom], 2),
+                "algorithmic_flops": dom_flops,
+                "peak_kind": f"{peak_kind}: {'2 x ' if fp8 else ''}bf16_tflops_sustained "
+                             f"(burst: {ratio * peaks['bf16_tflops']:.0f} TFLOP/s)"}
     step_weight_bytes = gemm1_bytes + gemm2_bytes
+    step_flops = gemm1_flops + gemm2_flops
     # cpu baseline: the oracle on the whole batch, once
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -406,6 +422,8 @@ def run_ours(args, rank, world, local_rank):
                      "achieved_gbs": round(step_weight_bytes / (ms_step / 1e3) / 1e9, 1),
                      "frac": round(step_weight_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                      "touched_experts": touched},
+        "step_tensor": {"flops": step_flops,
+                        "achieved_tflops": round(step_flops / (ms_step / 1e3) / 1e12, 1)},
         "kernels_us": {k: round(1e3 * v, 2) for k, v in kern_ms.items()},
         "plan": plan,
         "cpu_baseline": cpu,

@@ -122,8 +122,9 @@ FMOE_API const char* fused_moe_status_string(fmoe_status status);
  * invalid.  Host-only, makes no CUDA call. */
 FMOE_API size_t fused_moe_workspace_size(const fmoe_dims* dims);
 
-/* Zero the workspace header (status word included).  Call once on a new workspace
- * before its first use.  Asynchronous on `stream`. */
+/* Zero the workspace header (status word and routing counters).  Call once on a new
+ * workspace before its first use; the calls below leave the counters at zero.
+ * Asynchronous on `stream`. */
 FMOE_API fmoe_status fused_moe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream stream);
 
 /* Step 1, routing.

@@ -29,7 +29,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   bool fp8 = false, swap = false;
   int R = 0, chunk_rows = 0, max_chunks = 0, s1max = 0, s2max = 0;
-  size_t hdr = 0, amax_x = 0, amax_h = 0, chunks = 0;
+  size_t hdr = 0, counters = 0, amax_x = 0, amax_h = 0, chunks = 0, logits = 0;
   size_t ids = 0, tw = 0, counts = 0, offsets = 0, rows = 0, inv = 0;
   size_t x_in = 0, out_dev = 0, a_perm = 0, p1 = 0, h = 0, hq = 0, p2 = 0, y = 0;
   size_t total = 0;
@@ -79,7 +79,9 @@ Layout make_layout(const fmoe_dims& d) {
     return o;
   };
   L.hdr = take(sizeof(WsHeader));
+  L.counters = take(static_cast<size_t>(kRouterMaxTiles) * 4);  // zeroed with the header
   L.amax_x = take(static_cast<size_t>(std::max(T, 1)) * 4);
+  L.logits = take(static_cast<size_t>(T) * E * 4);
   L.amax_h = take(static_cast<size_t>(kAmaxSlots) * 4);
   L.chunks = take(static_cast<size_t>(L.max_chunks) * sizeof(Chunk));
   L.ids = take(static_cast<size_t>(R) * 4);
@@ -246,6 +248,8 @@ fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   a.topk_ids = ids;
   a.topk_w = tw;
   a.amax_part = reinterpret_cast<float*>(W + L.amax_x);
+  a.logits_g = reinterpret_cast<float*>(W + L.logits);
+  a.tile_counters = reinterpret_cast<int32_t*>(W + L.counters);
   a.hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   a.T = d.T;
   a.H = d.H;
@@ -321,7 +325,8 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
 
   const uint32_t xbox = swap ? 16u : 128u;
   GemmArgs g{};
-  if (!encode_map(&g.map_w, w13, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(E) * 2 * I, 128) ||
+  if (!encode_map(&g.map_w, w13, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(E) * 2 * I,
+                  swap ? 16u : 128u) ||
       !encode_map(&g.map_x, a_perm, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(R), xbox))
     return FMOE_ERR_CUDA;
   g.chunks = chunks;
@@ -329,7 +334,8 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g.hdr_w = hdr;
   g.status = &hdr->status;
   g.out = swap ? reinterpret_cast<float*>(W + L.p1) : (fp8 ? hbuf : nullptr);
-  g.out_bf16 = (!swap && !fp8) ? static_cast<uint16_t*>(hq) : nullptr;
+  g.out_bf16 = fp8 ? nullptr : static_cast<uint16_t*>(hq);
+  g.h_out = fp8 ? hbuf : nullptr;
   g.w_scale = fp8 ? sc->w13_scale : nullptr;
   g.topk_w = tw;
   g.sorted_rows = rows;
@@ -363,6 +369,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   if (fp8) {
     QuantHArgs q{};
     q.h = hbuf;
+    q.h_bf16 = nullptr;
     q.hq = static_cast<uint8_t*>(hq);
     q.amax_part = amax_h;
     q.hdr = hdr;
@@ -378,6 +385,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
     return FMOE_ERR_CUDA;
   g2.out = swap ? reinterpret_cast<float*>(W + L.p2) : y;
   g2.out_bf16 = nullptr;
+  g2.h_out = nullptr;
   g2.w_scale = fp8 ? sc->w2_scale : nullptr;
   g2.K = I;
   g2.Nout = H;
@@ -478,8 +486,9 @@ size_t fused_moe_workspace_size(const fmoe_dims* dims) {
 
 fmoe_status fused_moe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream stream) {
   if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
-  if (ws_bytes < sizeof(WsHeader)) return FMOE_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+  const size_t head = sizeof(WsHeader) + static_cast<size_t>(kRouterMaxTiles) * 4;
+  if (ws_bytes < head) return FMOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, head, static_cast<cudaStream_t>(stream)));
 }
 
 fmoe_status fused_moe_route(const fmoe_dims* dims, const void* x, const void* router_w,

@@ -52,9 +52,10 @@ __global__ void __launch_bounds__(kEwThreads) finalize1_kernel(Finalize1Args a) 
   __shared__ float red[kEwThreads / 32];
   griddep_wait();
   griddep_launch_dependents();
+  const int S = a.hdr->split1;
+  if (S == 1) return;  // the unsplit first contraction already wrote h and its max
   for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];
   __syncthreads();
-  const int S = a.hdr->split1;
   const float s1 = a.fp8 ? a.hdr->s1 : 1.f;
   const int I = a.I, I4 = a.I / 4;
   const size_t plane = static_cast<size_t>(a.R) * 2 * I;
@@ -137,8 +138,23 @@ __global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
   const size_t total = static_cast<size_t>(a.R) * a.I / 16;
   for (size_t v = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; v < total;
        v += static_cast<size_t>(gridDim.x) * kEwThreads) {
-    const float4* src = reinterpret_cast<const float4*>(a.h) + 4 * v;
-    const float4 f0 = src[0], f1 = src[1], f2 = src[2], f3 = src[3];
+    float4 f0, f1, f2, f3;
+    if (a.h_bf16 != nullptr) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.h_bf16) + 2 * v;
+      const uint4 b0 = src[0], b1 = src[1];
+      auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+      auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
+      f0 = make_float4(lo(b0.x), hi(b0.x), lo(b0.y), hi(b0.y));
+      f1 = make_float4(lo(b0.z), hi(b0.z), lo(b0.w), hi(b0.w));
+      f2 = make_float4(lo(b1.x), hi(b1.x), lo(b1.y), hi(b1.y));
+      f3 = make_float4(lo(b1.z), hi(b1.z), lo(b1.w), hi(b1.w));
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(a.h) + 4 * v;
+      f0 = src[0];
+      f1 = src[1];
+      f2 = src[2];
+      f3 = src[3];
+    }
     uint4 q;
     q.x = e4m3x4(f0.x * inv, f0.y * inv, f0.z * inv, f0.w * inv);
     q.y = e4m3x4(f1.x * inv, f1.y * inv, f1.z * inv, f1.w * inv);

@@ -47,17 +47,23 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 
 // ----------------------------------------------------------------------------- router
 struct RouterArgs {
-  const uint16_t* x;    // [T, H] bf16 bits
-  const uint16_t* wr;   // [E, H] bf16 bits
-  int32_t* topk_ids;    // [T, k]
-  float* topk_w;        // [T, k]
-  float* amax_part;     // [ceil(T / tokens_per_cta)] per-CTA max |x|
+  const uint16_t* x;       // [T, H] bf16 bits
+  const uint16_t* wr;      // [E, H] bf16 bits
+  int32_t* topk_ids;       // [T, k]
+  float* topk_w;           // [T, k]
+  float* amax_part;        // [token tiles] per-tile max |x|
+  float* logits_g;         // [T, E] logits when the experts are split over CTAs
+  int32_t* tile_counters;  // [kRouterMaxTiles] zero between calls (self-resetting)
   WsHeader* hdr;
   int T, H, E, k;
   int num_sms;
+  int experts_per_cta;     // set by the launcher
 };
+// Token tiles that may split their experts over several CTAs (counters in the header area).
+constexpr int kRouterMaxTiles = 4096;
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 int router_tokens_per_cta(int T, int H, int E, int num_sms);
+int router_experts_per_warp(int E);
 
 // ----------------------------------------------------------------------------- permute
 // How the grouped GEMMs are planned from the per-expert offsets.
@@ -109,13 +115,15 @@ struct PlanArgs {
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
 
 struct GemmArgs {
-  CUtensorMap map_w;       // weights [E * rows_per_expert, K], box {BK, 128}
+  CUtensorMap map_w;       // weights [E * rows_per_expert, K], box {BK, 128} (swap-AB
+                           // first contraction: box {BK, 16})
   CUtensorMap map_x;       // activations [R, K], box {BK, 16 (swap) or 128 (normal)}
   const Chunk* chunks;
   const WsHeader* hdr;
   int32_t* status;
   float* out;              // swap: partials [S][R][Nout]; normal: h [R, I] or y [R, H]
-  uint16_t* out_bf16;      // normal, first contraction, bf16 format: h rounded to bf16
+  uint16_t* out_bf16;      // first contraction, bf16 format: h rounded to bf16
+  float* h_out;            // swap-AB first contraction, FP8, split 1: h [R, I] fp32
   const float* w_scale;    // [E] per-expert weight scale (FP8) or null
   const float* topk_w;     // [R] flattened routing weights (normal, second contraction)
   const int32_t* sorted_rows;
@@ -146,7 +154,8 @@ struct Finalize1Args {
 cudaError_t launch_finalize1(const Finalize1Args& a, int num_sms, cudaStream_t s);
 
 struct QuantHArgs {
-  const float* h;           // [R, I]
+  const float* h;           // [R, I] fp32, or
+  const uint16_t* h_bf16;   // [R, I] bf16 (when non-null)
   uint8_t* hq;              // [R, I] e4m3
   const float* amax_part;
   WsHeader* hdr;

@@ -197,7 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       auto load_w = [&](int st, const Unit& t, int kb) {
         uint8_t* sa = smem + st * stage_bytes;
         const int kx = kb * kBK;
-        if (kSwap) {
+        if (kSwap && kGemm == 1) {
+          // 128 rows as four 32-row quarters: quarter q = 16 gate rows of features
+          // tile*64 + 16q .. +15, then the 16 matching up rows, so one warp's TMEM lanes
+          // hold both halves of its features
+          const int row = t.e * a.rows_per_expert + t.tile * 64;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tma_load_2d(sa + (32 * q) * 128, &a.map_w, &ctl.full[st], kx, row + 16 * q, pol_w);
+            tma_load_2d(sa + (32 * q + 16) * 128, &a.map_w, &ctl.full[st], kx, row + a.I + 16 * q,
+                        pol_w);
+          }
+        } else if (kSwap) {
           tma_load_2d(sa, &a.map_w, &ctl.full[st], kx, t.e * a.rows_per_expert + t.tile * 128, pol_w);
         } else {
           uint8_t* sb = sa + kTileA;
@@ -336,7 +347,46 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       tc_fence_after();
       const uint32_t tb =
           tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (kSwap) {
+      if constexpr (kSwap && kGemm == 1) {
+        // lane r of quarter q: gate (r%32 < 16) or up (r%32 >= 16) of feature
+        // tile*64 + 16q + r%16; column c = token row0 + c
+        const int ncols = ((t.nrows + 15) / 16) * 16;
+        const int f = t.tile * 64 + q * 16 + (lane & 15);
+        if (S == 1) {
+          // whole K in this tile: apply the scale and SiLU(g)*u here
+          const float sc = kFp8 ? a.hdr->s1 * a.w_scale[t.e] : 1.f;
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float v[16];
+            tmem_ld16(tb + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float up = __shfl_xor_sync(0xffffffffu, v[i], 16);
+              if (lane < 16 && c0 + i < t.nrows) {
+                const float h = silu_f(v[i] * sc) * (up * sc);
+                const size_t o = static_cast<size_t>(t.row0 + c0 + i) * a.I + f;
+                if constexpr (kFp8) {
+                  a.h_out[o] = h;
+                  amax = fmaxf(amax, fabsf(h));
+                } else {
+                  a.out_bf16[o] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                }
+              }
+            }
+          }
+        } else {
+          const int feat = (lane & 16) ? a.I + f : f;
+          float* dst = a.out + (static_cast<size_t>(t.s) * a.R + t.row0) * a.Nout + feat;
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float v[16];
+            tmem_ld16(tb + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < t.nrows) dst[static_cast<size_t>(c0 + i) * a.Nout] = v[i];
+          }
+        }
+      } else if constexpr (kSwap) {
         // lane r = output feature tile*128 + r, column c = token row0 + c
         const int ncols = ((t.nrows + 15) / 16) * 16;
         float* dst = a.out + (static_cast<size_t>(t.s) * a.R + t.row0) * a.Nout + t.tile * 128 + r;
@@ -362,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i] * sc) * (up[i] * sc);
           if (valid) {
             if constexpr (kFp8) {
+              // fp32 h for the per-tensor re-quantisation (quant_h); storing it rounded
+              // to bf16 would double-round a few percent of the e4m3 codes
               float4* dst = reinterpret_cast<float4*>(a.out + o + c0);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -370,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                                          fmaxf(fabsf(h[4 * i + 2]), fabsf(h[4 * i + 3]))));
               }
             } else {
+              // bf16 format: h rounded to bf16 is the second contraction's input
               uint32_t pk[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
@@ -412,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         acc_phase ^= 1u;
       }
     }
-    if constexpr (!kSwap && kGemm == 1 && kFp8) {
+    if constexpr (kGemm == 1 && kFp8) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       if (lane == 0) atomicMax(&ctl.amax_bits, __float_as_int(amax));
@@ -420,8 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   }
 
   __syncthreads();
-  if constexpr (!kSwap && kGemm == 1 && kFp8) {
-    if (threadIdx.x == 0) {
+  // per-CTA max |h| when this kernel produced h (normal variant, or swap-AB unsplit)
+  if constexpr (kGemm == 1 && kFp8) {
+    if (threadIdx.x == 0 && (!kSwap || S == 1)) {
       a.amax_part[blockIdx.x] = __int_as_float(ctl.amax_bits);
       if (blockIdx.x == 0) a.hdr_w->amax_h_count = gridDim.x;
     }

@@ -107,22 +107,59 @@ __device__ void build_plan(const int* offsets, int E, int R, const PlanParams& p
 }
 
 
+// Stable grouping in one CTA: warp w owns the contiguous segment of routed rows
+// [w*seg, (w+1)*seg).  Pass 1 counts each warp's rows per expert, the counts give the
+// offsets and each (expert, warp) start position, and pass 2 walks every segment again
+// in ascending order, so rows of one expert keep their flattened order (t*k+j).
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
+  constexpr int kWarps = kPermThreads / 32;
   __shared__ int cnt[kMaxExperts];
   __shared__ int base[kMaxExperts + 1];
-  __shared__ int ctot[kMaxExperts];
-  __shared__ int wc[kPermThreads / 32][kMaxExperts];
+  __shared__ int wc[kWarps][kMaxExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, R = a.R;
+  const int seg = (R + kWarps - 1) / kWarps;
+  const int lo = min(R, warp * seg), hi = min(R, lo + seg);
 
-  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  for (int i = tid; i < kWarps * E; i += kPermThreads) wc[i / E][i % E] = 0;
   griddep_wait();
   griddep_launch_dependents();
   __syncthreads();
-  for (int i = tid; i < R; i += kPermThreads) {
-    const int e = a.topk_ids[i];
-    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
-    else record_status(&a.hdr->status, ST_BOUNDS);
+
+  // The ids of a warp's segment are read kBatch*32 at a time (kBatch loads in flight
+  // per lane), then handled 32 at a time in ascending order.
+  constexpr int kBatch = 8;
+  auto load_batch = [&](int i0, int (&ev)[kBatch]) {
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = i0 + 32 * j + lane;
+      int e = i < hi ? a.topk_ids[i] : E;
+      if (i < hi && (e < 0 || e >= E)) {
+        record_status(&a.hdr->status, ST_BOUNDS);
+        e = E + 1;  // invalid: matches only other invalid lanes, never placed
+      }
+      ev[j] = e;
+    }
+  };
+
+  // pass 1: rows per (warp, expert)
+  for (int i0 = lo; i0 < hi; i0 += 32 * kBatch) {
+    int ev[kBatch];
+    load_batch(i0, ev);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (i0 + 32 * j >= hi) break;  // warp-uniform
+      const int e = ev[j];
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e < E && lane == __ffs(peers) - 1) wc[warp][e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kPermThreads) {
+    int c = 0;
+    for (int w = 0; w < kWarps; ++w) c += wc[w][e];
+    cnt[e] = c;
   }
   __syncthreads();
 
@@ -157,11 +194,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
       base[E] = incl;
     }
   }
-  if (tid == 32) {
-    // activation scale from the router's per-CTA maxima
+  if (warp == 1) {
+    // activation scale from the router's per-tile maxima (one warp, strided)
     float amax = 0.f;
     const int n = a.hdr->router_ctas;
-    for (int i = 0; i < n; ++i) amax = fmaxf(amax, a.amax_part[i]);
+    for (int i = lane; i < n; i += 32) amax = fmaxf(amax, a.amax_part[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     float s1 = 1.f, inv1 = 1.f;
     if (a.fp8) {
       if (a.a1_static > 0.f) {
@@ -172,44 +211,45 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
         inv1 = 448.0f / amax;
       }
     }
-    a.hdr->amax_x = amax;
-    a.hdr->s1 = s1;
-    a.hdr->inv1 = inv1;
+    if (lane == 0) {
+      a.hdr->amax_x = amax;
+      a.hdr->s1 = s1;
+      a.hdr->inv1 = inv1;
+    }
   }
   __syncthreads();
   if (a.with_plan && warp == 0) build_plan(base, E, R, a.plan, a.hdr);
+  // first position of each (warp, expert)
+  for (int e = tid; e < E; e += kPermThreads) {
+    int run = base[e];
+    for (int w = 0; w < kWarps; ++w) {
+      const int v = wc[w][e];
+      wc[w][e] = run;
+      run += v;
+    }
+  }
   __syncthreads();
 
-  // stable ranks, kPermThreads entries at a time
-  for (int c0 = 0; c0 < R; c0 += kPermThreads) {
-    for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) wc[i / E][i % E] = 0;
-    __syncthreads();
-    const int i = c0 + tid;
-    int e = i < R ? a.topk_ids[i] : E;
-    const bool valid = e >= 0 && e < E;
-    if (!valid) e = E;  // sentinel: matches only other invalid lanes
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (valid && lane == __ffs(peers) - 1) wc[warp][e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += kPermThreads) {
-      int run = 0;
-      for (int w = 0; w < kPermThreads / 32; ++w) {
-        const int v = wc[w][ee];
-        wc[w][ee] = run;
-        run += v;
+  // pass 2: place every row, in ascending order within each warp's segment
+  for (int i0 = lo; i0 < hi; i0 += 32 * kBatch) {
+    int ev[kBatch];
+    load_batch(i0, ev);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (i0 + 32 * j >= hi) break;  // warp-uniform
+      const int i = i0 + 32 * j + lane;
+      const int e = ev[j];
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (e < E) {
+        const int pos = wc[warp][e] + rank;
+        a.sorted_rows[pos] = i;
+        a.inv_perm[i] = pos;
       }
-      ctot[ee] = run;
+      __syncwarp();
+      if (e < E && lane == __ffs(peers) - 1) wc[warp][e] += __popc(peers);
+      __syncwarp();
     }
-    __syncthreads();
-    if (valid) {
-      const int pos = base[e] + wc[warp][e] + rank;
-      a.sorted_rows[pos] = i;
-      a.inv_perm[i] = pos;
-    }
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += kPermThreads) base[ee] += ctot[ee];
-    __syncthreads();
   }
 }
 

@@ -28,16 +28,13 @@ namespace {
 
 constexpr int kRouterThreads = 256;
 
-__device__ __forceinline__ void fma8_bf16(float& acc, const uint4& xa, const uint4& wa) {
-  const uint32_t xs[4] = {xa.x, xa.y, xa.z, xa.w};
-  const uint32_t ws[4] = {wa.x, wa.y, wa.z, wa.w};
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  // element 2i sits in the low half of word i, element 2i+1 in the high half
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // element 2i sits in the low half, element 2i+1 in the high half
-    const float x0 = __uint_as_float(xs[i] << 16), x1 = __uint_as_float(xs[i] & 0xFFFF0000u);
-    const float w0 = __uint_as_float(ws[i] << 16), w1 = __uint_as_float(ws[i] & 0xFFFF0000u);
-    acc = __fmaf_rn(x0, w0, acc);
-    acc = __fmaf_rn(x1, w1, acc);
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
 
@@ -46,16 +43,19 @@ __device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
 }
 
 template <int TB, int EG>
-__global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
+__global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                    // [TB][H]
   float* logits = reinterpret_cast<float*>(smem + TB * a.H * 2);       // [TB][E]
   __shared__ float red[kRouterThreads / 32];
+  __shared__ int is_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * TB;
+  const int tile = blockIdx.x, group = blockIdx.y;
+  const int t0 = tile * TB;
   const int H = a.H, E = a.E;
   const int vec_per_row = H / 8;  // 16-byte vectors per row
+  const bool split = gridDim.y > 1;
 
   griddep_wait();
   griddep_launch_dependents();
@@ -79,34 +79,66 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   if (lane == 0) red[warp] = amax;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && group == 0) {
     float m = 0.f;
     for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, red[w]);
-    a.amax_part[blockIdx.x] = m;
-    if (blockIdx.x == 0) a.hdr->router_ctas = gridDim.x;
+    a.amax_part[tile] = m;
+    if (tile == 0) a.hdr->router_ctas = gridDim.x;
   }
 
-  // ---- logits in the canonical order
+  // ---- logits of this CTA's experts, in the canonical order
   const int steps = H / 256;  // chunks per lane
-  for (int eb = warp * EG; eb < E; eb += (kRouterThreads / 32) * EG) {
+  const int e_begin = group * a.experts_per_cta;
+  const int e_end = min(E, e_begin + a.experts_per_cta);
+  constexpr int U = 2;  // chunk steps whose router rows are loaded together
+  // Accumulators acc[t][g] are updated in pairs with one paired FMA (each component
+  // rounds exactly like a scalar fmaf), element by element in ascending order, so
+  // every logit keeps the canonical summation order.
+  constexpr int NACC = TB * EG;
+  constexpr bool kPairG = (EG % 2 == 0);  // pairs (t, g), (t, g+1); else (t, g), (t+1, g)
+  for (int eb = e_begin + warp * EG; eb < e_end; eb += (kRouterThreads / 32) * EG) {
     float acc[TB][EG];
 #pragma unroll
     for (int t = 0; t < TB; ++t)
 #pragma unroll
       for (int g = 0; g < EG; ++g) acc[t][g] = 0.f;
-    for (int s = 0; s < steps; ++s) {
-      const int chunk = lane + 32 * s;
-      uint4 wv[EG];
+    for (int s0 = 0; s0 < steps; s0 += U) {
+      uint4 wv[U][EG];
 #pragma unroll
-      for (int g = 0; g < EG; ++g) {
-        const int e = min(eb + g, E - 1);
-        wv[g] = __ldg(reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H) + chunk);
-      }
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int t = 0; t < TB; ++t) {
-        const uint4 xv = reinterpret_cast<const uint4*>(xs + t * H)[chunk];
+        for (int g = 0; g < EG; ++g) {
+          const int e = min(eb + g, e_end - 1);
+          const int chunk = lane + 32 * min(s0 + u, steps - 1);
+          wv[u][g] = __ldg(reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H) + chunk);
+        }
 #pragma unroll
-        for (int g = 0; g < EG; ++g) fma8_bf16(acc[t][g], xv, wv[g]);
+      for (int u = 0; u < U; ++u) {
+        if (s0 + u < steps) {
+          const int chunk = lane + 32 * (s0 + u);
+          float wf[EG][8], xf[TB][8];
+#pragma unroll
+          for (int g = 0; g < EG; ++g) unpack8(wv[u][g], wf[g]);
+#pragma unroll
+          for (int t = 0; t < TB; ++t) unpack8(reinterpret_cast<const uint4*>(xs + t * H)[chunk], xf[t]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if constexpr (NACC % 2 == 0) {
+#pragma unroll
+              for (int m = 0; m < NACC; m += 2) {
+                const int ta = m / EG, ga = m % EG;
+                const int tb = kPairG ? ta : ta + 1, gb = kPairG ? ga + 1 : ga;
+                const float2 r = __ffma2_rn(make_float2(xf[ta][i], xf[tb][i]),
+                                            make_float2(wf[ga][i], wf[gb][i]),
+                                            make_float2(acc[ta][ga], acc[tb][gb]));
+                acc[ta][ga] = r.x;
+                acc[tb][gb] = r.y;
+              }
+            } else {
+              acc[0][0] = __fmaf_rn(xf[0][i], wf[0][i], acc[0][0]);
+            }
+          }
+        }
       }
     }
 #pragma unroll
@@ -116,8 +148,35 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
         float p = acc[t][g];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) p = p + __shfl_xor_sync(0xffffffffu, p, off);
-        if (lane == 0 && eb + g < E) logits[t * E + eb + g] = p;
+        if (lane == 0 && eb + g < e_end) {
+          if (split) {
+            if (t0 + t < a.T) a.logits_g[static_cast<size_t>(t0 + t) * E + eb + g] = p;
+          } else {
+            logits[t * E + eb + g] = p;
+          }
+        }
       }
+  }
+
+  if (split) {
+    // The last of the gridDim.y CTAs of this token tile to finish picks the top-k
+    // (counter reset for the next call by that CTA).
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const int prev = atomicAdd(&a.tile_counters[tile], 1);
+      is_last = prev == static_cast<int>(gridDim.y) - 1;
+      if (is_last) {
+        a.tile_counters[tile] = 0;
+        __threadfence();
+      }
+    }
+    __syncthreads();
+    if (!is_last) return;
+    for (int i = threadIdx.x; i < TB * E; i += kRouterThreads) {
+      const int t = i / E, e = i % E;
+      logits[i] = (t0 + t < a.T) ? __ldcg(a.logits_g + static_cast<size_t>(t0 + t) * E + e) : 0.f;
+    }
   }
   __syncthreads();
 
@@ -167,28 +226,42 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
 }
 
 template <int TB, int EG>
-cudaError_t launch_tb(const RouterArgs& a, cudaStream_t s) {
+cudaError_t launch_tb(RouterArgs a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(TB) * a.H * 2 + static_cast<size_t>(TB) * a.E * 4;
   cudaError_t err = set_max_dynamic_smem<router_kernel<TB, EG>>(160 * 1024);
   if (err != cudaSuccess) return err;
-  const int grid = (a.T + TB - 1) / TB;
-  return launch_k(router_kernel<TB, EG>, dim3(grid), dim3(kRouterThreads), smem, s, a);
+  // favour shared memory over L1 so that two CTAs fit per SM
+  cudaFuncSetAttribute(router_kernel<TB, EG>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  const int tiles = (a.T + TB - 1) / TB;
+  const int per_cta = (kRouterThreads / 32) * EG;
+  int groups = (a.E + per_cta - 1) / per_cta;
+  if (tiles > kRouterMaxTiles) groups = 1;  // no tile counters for that many tiles
+  a.experts_per_cta = groups == 1 ? a.E : per_cta;
+  return launch_k(router_kernel<TB, EG>, dim3(tiles, groups), dim3(kRouterThreads), smem, s, a);
 }
 
 template <int TB>
 cudaError_t launch_eg(const RouterArgs& a, cudaStream_t s) {
-  if (a.E >= 128) return launch_tb<TB, 4>(a, s);
-  if (a.E >= 16) return launch_tb<TB, 2>(a, s);
+  const int eg = router_experts_per_warp(a.E);
+  if (eg == 4) return launch_tb<TB, 4>(a, s);
+  if (eg == 2) return launch_tb<TB, 2>(a, s);
   return launch_tb<TB, 1>(a, s);
 }
 
 }  // namespace
 
+int router_experts_per_warp(int E) { return E >= 128 ? 4 : (E >= 16 ? 2 : 1); }
+
+// Tokens per CTA: the largest of 4, 2, 1 that still gives at least two CTAs per SM
+// (counting the expert groups), else 1.
 int router_tokens_per_cta(int T, int H, int E, int num_sms) {
   (void)H;
-  (void)E;
-  if (T >= 8 * num_sms) return 4;
-  if (T >= 2 * num_sms) return 2;
+  const int per_cta = (kRouterThreads / 32) * router_experts_per_warp(E);
+  const int groups = (E + per_cta - 1) / per_cta;
+  for (int tb : {4, 2}) {
+    const long ctas = static_cast<long>((T + tb - 1) / tb) * groups;
+    if (ctas >= 2L * num_sms) return tb;
+  }
   return 1;
 }
 

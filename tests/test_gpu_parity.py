@@ -252,3 +252,35 @@ def test_full_size_matches_oracle(full_weights, workload, T):
         other = "normal" if (s.R + s.E - 1) // s.E <= 64 else "swap_ab"
         out_o, _ = run_fused(inp, g, other)
         assert max_rel_err(bf16_bits_to_float(out_o), bf16_bits_to_float(ref["out"])) <= TOL["fp8"]
+
+
+ROUTER_SHAPES = [("mixtral_fp8_decode", T) for T in (1, 64)] + \
+                [("dsv3_fp8_decode", T) for T in (16, 256)] + \
+                [("swapab_adversarial_fp8", 8), ("prefill_fp8", 4096)]
+
+
+@pytest.mark.parametrize("workload,T", ROUTER_SHAPES, ids=[f"{w}-T{t}" for w, t in ROUTER_SHAPES])
+def test_router_full_shapes(workload, T):
+    """Routing and permutation alone at each workload's real (T, H, E, k), in the launch
+    configuration of the full layer: bit-exact ids, counts and permutation."""
+    s = minp.shape(workload, T)
+    x, wr = minp.make_activations(s, seed=0)
+    ids_ref, w_ref, _ = O.router(minp.bf16_bits(x), minp.bf16_bits(wr), s.top_k)
+    counts_ref, offs_ref, rows_ref, inv_ref = O.permute(ids_ref, s.E)
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, True)
+    ws = capi.alloc_workspace(dims)
+    R = s.R
+    ids = torch.empty(R, dtype=torch.int32, device="cuda")
+    tw = torch.empty(R, dtype=torch.float32, device="cuda")
+    bufs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (s.E, s.E + 1, R, R)]
+    a_perm = torch.empty(R, s.H, dtype=torch.uint8, device="cuda")
+    xd = x.cuda()
+    for _ in range(2):  # the second call starts from the counters the first one left
+        capi.fused_moe_route(dims, xd, wr.cuda(), ids, tw, ws)
+        capi.fused_moe_permute(dims, ids, xd, None, *bufs, a_perm, ws)
+        torch.cuda.synchronize()
+        assert capi.fused_moe_get_device_status(ws) == capi.FMOE_OK
+        assert np.array_equal(ids.cpu().numpy().reshape(s.T, s.top_k), ids_ref)
+        assert np.allclose(tw.cpu().numpy().reshape(s.T, s.top_k), w_ref, rtol=1e-6, atol=1e-9)
+        for got, ref in zip(bufs, (counts_ref, offs_ref, rows_ref, inv_ref)):
+            assert np.array_equal(got.cpu().numpy(), ref)
