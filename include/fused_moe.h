@@ -35,8 +35,9 @@
  *    asynchronously on it; results are valid once the stream reaches that point.
  *  - Argument checks run before any CUDA call and return synchronously:
  *      FMOE_ERR_INVALID_ARG  null dims / pointer, T < 0, H, I < 1, E < 1 or > 256,
- *                            top_k < 1 or > E, unknown wdtype / variant, FP8 without
- *                            weight scales
+ *                            top_k < 1 or > E, unknown wdtype / variant / routing
+ *                            mode, routing parameters outside their ranges, FP8
+ *                            without weight scales
  *      FMOE_ERR_UNSUPPORTED  H % 256 != 0, I % 128 != 0, H > 16384, a device pointer
  *                            not 16-byte aligned, sizes whose element counts exceed
  *                            2^31
@@ -62,7 +63,7 @@
 extern "C" {
 #endif
 
-#define FUSED_MOE_ABI_VERSION 1
+#define FUSED_MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FMOE_API __attribute__((visibility("default")))
@@ -93,6 +94,26 @@ typedef enum {
  * fp32 summation order. */
 typedef enum { FMOE_VARIANT_AUTO = 0, FMOE_VARIANT_SWAP_AB = 1, FMOE_VARIANT_NORMAL = 2 } fmoe_variant;
 
+/* How tokens choose experts.
+ *  FMOE_ROUTE_SOFTMAX: the k largest logits; weights = softmax over all E experts
+ *    renormalised over the k chosen.
+ *  FMOE_ROUTE_SIGMOID_GROUPED: the group-limited router of DeepSeek-V3 (the pages name
+ *    the model but not its router; this follows its published design):
+ *    s = fp32(sigmoid(logit)) (evaluated in fp64, rounded once), sb = s + bias[e] (fp32);
+ *    the E experts form n_group groups of E/n_group consecutive experts, a group scores
+ *    the sum of its two largest sb, the topk_group best groups are kept (ties to the
+ *    lower group), then the k largest sb inside them (ties to the lower expert);
+ *    weights = s / (sum of the chosen s) * routed_scaling. */
+typedef enum { FMOE_ROUTE_SOFTMAX = 0, FMOE_ROUTE_SIGMOID_GROUPED = 1 } fmoe_route_mode;
+
+typedef struct {
+  int32_t mode;           /* fmoe_route_mode */
+  int32_t n_group;        /* SIGMOID_GROUPED: 1..32 groups, E % n_group == 0, E/n_group >= 2 */
+  int32_t topk_group;     /* SIGMOID_GROUPED: 1..n_group, topk_group * E/n_group >= top_k */
+  float routed_scaling;   /* SIGMOID_GROUPED: > 0, multiplies the renormalised weights */
+  const float* bias;      /* SIGMOID_GROUPED: [E] device fp32 selection bias, or NULL */
+} fmoe_routing;
+
 typedef struct {
   int32_t T;        /* tokens */
   int32_t H;        /* hidden size */
@@ -101,6 +122,7 @@ typedef struct {
   int32_t top_k;    /* experts per token */
   int32_t wdtype;   /* fmoe_wdtype */
   int32_t variant;  /* fmoe_variant */
+  const fmoe_routing* routing; /* host pointer, read during the call; NULL = softmax */
 } fmoe_dims;
 
 typedef struct {
@@ -193,8 +215,10 @@ FMOE_API fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host
                               const void* w13, const void* w2, const fmoe_scales* scales,
                               void* out_host, void* ws, size_t ws_bytes, fmoe_stream stream);
 
-/* Number of kernels one fused_moe call launches for these dims (FP8: 7 NORMAL, 8
- * SWAP_AB; bf16: 6 NORMAL, 7 SWAP_AB; 0 for T == 0; -1 for invalid dims).  Host-only. */
+/* Number of kernels one fused_moe call launches for these dims: router, gemm1,
+ * finalize1 (SWAP_AB only), quant_h (FP8 only), gemm2 and combine, plus permute and
+ * gather unless the router runs them (T*k <= 2048; the gather only when
+ * T*k*H*2 <= 128 KB).  0 for T == 0, -1 for invalid dims.  Host-only. */
 FMOE_API int32_t fused_moe_launches_per_call(const fmoe_dims* dims);
 
 /* Measurement: runs fused_moe once with a CUDA event recorded on `stream` before the
@@ -234,6 +258,14 @@ FMOE_API fmoe_status fused_moe_static_workspace(const fmoe_dims* dims, const voi
                                                 const void* w2, const fmoe_scales* scales,
                                                 void* out, int32_t* device_status,
                                                 fmoe_stream stream);
+
+/* Test of the device-side failure path: launches one warp that waits on an mbarrier
+ * nothing ever arrives at, with the same bounded wait every kernel of the library
+ * uses, limited to budget_ns (at most 10 s).  The wait gives up, records
+ * FMOE_ERR_TIMEOUT in the workspace status word and the kernel returns normally, so
+ * the CUDA context stays usable.  Asynchronous on `stream`. */
+FMOE_API fmoe_status fused_moe_selftest_wait(void* ws, size_t ws_bytes, uint64_t budget_ns,
+                                             fmoe_stream stream);
 
 /* Synchronous: waits for `stream`, then returns the sticky device status recorded in
  * ws (FMOE_OK, FMOE_ERR_TIMEOUT or FMOE_ERR_DEVICE_BOUNDS), or FMOE_ERR_CUDA if the

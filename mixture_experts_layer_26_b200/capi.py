@@ -36,14 +36,23 @@ EXPORTED = (
     "fused_moe_workspace_init", "fused_moe_route", "fused_moe_permute", "fused_moe_experts",
     "fused_moe_combine", "fused_moe", "fused_moe_host_io", "fused_moe_get_device_status",
     "fused_moe_debug_scalars", "fused_moe_launches_per_call", "fused_moe_profile",
-    "fused_moe_static_workspace",
+    "fused_moe_static_workspace", "fused_moe_selftest_wait",
 )
 STATIC_WS_BYTES = 64 << 20  # FUSED_MOE_STATIC_WS_BYTES
 
 
+FMOE_ROUTE_SOFTMAX, FMOE_ROUTE_SIGMOID_GROUPED = 0, 1
+
+
+class FmoeRouting(ctypes.Structure):
+    _fields_ = [("mode", c_int32), ("n_group", c_int32), ("topk_group", c_int32),
+                ("routed_scaling", c_float), ("bias", c_void_p)]
+
+
 class FmoeDims(ctypes.Structure):
     _fields_ = [("T", c_int32), ("H", c_int32), ("I", c_int32), ("E", c_int32),
-                ("top_k", c_int32), ("wdtype", c_int32), ("variant", c_int32)]
+                ("top_k", c_int32), ("wdtype", c_int32), ("variant", c_int32),
+                ("routing", POINTER(FmoeRouting))]
 
 
 class FmoeScales(ctypes.Structure):
@@ -79,6 +88,8 @@ _dev_status = _sig("fused_moe_get_device_status", c_int32, c_void_p, c_void_p)
 _dbg = _sig("fused_moe_debug_scalars", c_int32, c_void_p, POINTER(c_float), POINTER(c_int32),
             c_void_p)
 _launches = _sig("fused_moe_launches_per_call", c_int32, _DP)
+_selftest_wait = _sig("fused_moe_selftest_wait", c_int32, c_void_p, c_size_t, ctypes.c_uint64,
+                      c_void_p)
 _static_ws = _sig("fused_moe_static_workspace", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p,
                   _SP, c_void_p, c_void_p, c_void_p)
 _profile = _sig("fused_moe_profile", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
@@ -116,8 +127,21 @@ def _stream(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
-def make_dims(T: int, H: int, I: int, E: int, top_k: int, fp8: bool, variant: str = "auto") -> FmoeDims:
-    return FmoeDims(T, H, I, E, top_k, FMOE_FP8_E4M3 if fp8 else FMOE_BF16, VARIANTS[variant])
+def make_routing(n_group: int, topk_group: int, routed_scaling: float = 1.0,
+                 bias: Optional[torch.Tensor] = None) -> FmoeRouting:
+    """Group-limited sigmoid routing (DeepSeek-V3 style); bias: [E] fp32 device tensor."""
+    r = FmoeRouting(FMOE_ROUTE_SIGMOID_GROUPED, n_group, topk_group, float(routed_scaling),
+                    _ptr(bias))
+    r._bias_ref = bias  # keep the tensor alive with the descriptor
+    return r
+
+
+def make_dims(T: int, H: int, I: int, E: int, top_k: int, fp8: bool, variant: str = "auto",
+              routing: Optional[FmoeRouting] = None) -> FmoeDims:
+    d = FmoeDims(T, H, I, E, top_k, FMOE_FP8_E4M3 if fp8 else FMOE_BF16, VARIANTS[variant],
+                 ctypes.pointer(routing) if routing is not None else None)
+    d._routing_ref = routing  # the C struct holds a raw pointer to it
+    return d
 
 
 def dims_of(x: torch.Tensor, w13: torch.Tensor, top_k: int, variant: str = "auto") -> FmoeDims:
@@ -215,6 +239,12 @@ def fused_moe_static_workspace(dims, x, router_w, w13, w2, scales, out, device_s
     st = _static_ws(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(w13), _ptr(w2), sp,
                     _ptr(out), _ptr(device_status), _stream(stream))
     return _check(st, "fused_moe_static_workspace") if check else st
+
+
+def fused_moe_selftest_wait(ws, budget_ns: int, stream=None, check=True) -> int:
+    """A bounded wait that must run out (records FMOE_ERR_TIMEOUT in ws)."""
+    st = _selftest_wait(_ptr(ws), ws.numel(), int(budget_ns), _stream(stream))
+    return _check(st, "fused_moe_selftest_wait") if check else st
 
 
 def fused_moe_launches_per_call(dims) -> int:

@@ -43,6 +43,21 @@ fmoe_status check_dims(const fmoe_dims* d) {
   if (d->wdtype != FMOE_BF16 && d->wdtype != FMOE_FP8_E4M3) return FMOE_ERR_INVALID_ARG;
   if (d->variant < FMOE_VARIANT_AUTO || d->variant > FMOE_VARIANT_NORMAL)
     return FMOE_ERR_INVALID_ARG;
+  if (d->routing != nullptr) {
+    const fmoe_routing& r = *d->routing;
+    if (r.mode != FMOE_ROUTE_SOFTMAX && r.mode != FMOE_ROUTE_SIGMOID_GROUPED)
+      return FMOE_ERR_INVALID_ARG;
+    if (r.mode == FMOE_ROUTE_SIGMOID_GROUPED) {
+      if (r.n_group < 1 || r.n_group > 32 || d->E % r.n_group != 0 || d->E / r.n_group < 2)
+        return FMOE_ERR_INVALID_ARG;
+      if (r.topk_group < 1 || r.topk_group > r.n_group ||
+          static_cast<int64_t>(r.topk_group) * (d->E / r.n_group) < d->top_k)
+        return FMOE_ERR_INVALID_ARG;
+      if (!(r.routed_scaling > 0.f) || r.routed_scaling > 1e30f) return FMOE_ERR_INVALID_ARG;
+      if (r.bias != nullptr && (reinterpret_cast<uintptr_t>(r.bias) & 3u) != 0)
+        return FMOE_ERR_UNSUPPORTED;
+    }
+  }
   if (d->H % 256 != 0 || d->I % 128 != 0 || d->H > 16384) return FMOE_ERR_UNSUPPORTED;
   const int64_t R = static_cast<int64_t>(d->T) * d->top_k;
   const int64_t lim = int64_t(1) << 31;
@@ -240,8 +255,22 @@ PlanParams plan_params(const fmoe_dims& d, const Layout& L, char* W) {
   return p;
 }
 
+// Small batches whose routed rows fit one CTA's permutation: the router's final CTA
+// also runs permute (+ plan) and, when the gathered rows are at most 128 KB, the gather.
+bool fuse_route_permute(const Layout& L) { return L.R <= 2048; }
+bool fuse_route_gather(const fmoe_dims& d, const Layout& L) {
+  return fuse_route_permute(L) && static_cast<size_t>(L.R) * d.H * 2 <= (size_t(128) << 10);
+}
+
+PermuteArgs permute_args(const fmoe_dims& d, const Layout& L, const int32_t* ids,
+                         const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
+                         int32_t* inv, char* W, bool with_plan);
+GatherArgs gather_args(const fmoe_dims& d, const Layout& L, const void* x, const int32_t* rows,
+                       void* a_perm, char* W);
+
 fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
-                       int32_t* ids, float* tw, char* W, cudaStream_t s) {
+                       int32_t* ids, float* tw, char* W, cudaStream_t s,
+                       const PermuteArgs* fused_perm = nullptr, const GatherArgs* fused_gather = nullptr) {
   RouterArgs a{};
   a.x = static_cast<const uint16_t*>(x);
   a.wr = static_cast<const uint16_t*>(rw);
@@ -256,14 +285,33 @@ fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   a.E = d.E;
   a.k = d.top_k;
   a.num_sms = num_sms();
-  FMOE_LAUNCH("router", launch_router(a, s), s);
+  a.mode = FMOE_ROUTE_SOFTMAX;
+  a.routed_scaling = 1.f;
+  if (d.routing != nullptr && d.routing->mode == FMOE_ROUTE_SIGMOID_GROUPED) {
+    a.mode = FMOE_ROUTE_SIGMOID_GROUPED;
+    a.n_group = d.routing->n_group;
+    a.topk_group = d.routing->topk_group;
+    a.routed_scaling = d.routing->routed_scaling;
+    a.bias = d.routing->bias;
+  }
+  a.route_done = &reinterpret_cast<WsHeader*>(W + L.hdr)->route_done;
+  if (fused_perm != nullptr) {
+    a.fuse_permute = 1;
+    a.perm = *fused_perm;
+    if (fused_gather != nullptr) {
+      a.fuse_gather = 1;
+      a.gather = *fused_gather;
+    }
+  }
+  FMOE_LAUNCH(fused_perm == nullptr ? "router"
+                                    : (fused_gather == nullptr ? "router_permute" : "router_permute_gather"),
+              launch_router(a, s), s);
   return FMOE_OK;
 }
 
-fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids, const void* x,
+PermuteArgs permute_args(const fmoe_dims& d, const Layout& L, const int32_t* ids,
                          const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
-                         int32_t* inv, void* a_perm, char* W, cudaStream_t s, bool with_plan) {
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+                         int32_t* inv, char* W, bool with_plan) {
   PermuteArgs p{};
   p.topk_ids = ids;
   p.counts = counts;
@@ -271,7 +319,7 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   p.sorted_rows = rows;
   p.inv_perm = inv;
   p.amax_part = reinterpret_cast<const float*>(W + L.amax_x);
-  p.hdr = hdr;
+  p.hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   p.R = L.R;
   p.E = d.E;
   p.k = d.top_k;
@@ -279,7 +327,12 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   p.a1_static = sc != nullptr ? sc->a1_scale : 0.f;
   p.with_plan = with_plan ? 1 : 0;
   p.plan = plan_params(d, L, W);
-  FMOE_LAUNCH(with_plan ? "permute_plan" : "permute", launch_permute(p, s), s);
+  return p;
+}
+
+GatherArgs gather_args(const fmoe_dims& d, const Layout& L, const void* x, const int32_t* rows,
+                       void* a_perm, char* W) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   GatherArgs g{};
   g.x = static_cast<const uint16_t*>(x);
   g.sorted_rows = rows;
@@ -289,7 +342,16 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   g.R = L.R;
   g.H = d.H;
   g.k = d.top_k;
-  g.fp8 = p.fp8;
+  g.fp8 = L.fp8 ? 1 : 0;
+  return g;
+}
+
+fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids, const void* x,
+                         const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
+                         int32_t* inv, void* a_perm, char* W, cudaStream_t s, bool with_plan) {
+  const PermuteArgs p = permute_args(d, L, ids, sc, counts, offsets, rows, inv, W, with_plan);
+  FMOE_LAUNCH(with_plan ? "permute_plan" : "permute", launch_permute(p, s), s);
+  const GatherArgs g = gather_args(d, L, x, rows, a_perm, W);
   FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
   return FMOE_OK;
 }
@@ -352,6 +414,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   FMOE_LAUNCH(swap ? "gemm1_swapab" : "gemm1_normal", launch_gemm(g, fp8, swap, 1, sms, s), s);
 
   if (swap) {
+    // split-K > 1: finish h from the partials (returns at once when the plan chose split 1)
     Finalize1Args f{};
     f.part = reinterpret_cast<const float*>(W + L.p1);
     f.offsets = offsets;
@@ -449,9 +512,17 @@ fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   int32_t* rows = reinterpret_cast<int32_t*>(W + L.rows);
   int32_t* inv = reinterpret_cast<int32_t*>(W + L.inv);
   float* y = reinterpret_cast<float*>(W + L.y);
-  FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
-  FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s,
-                        /*with_plan=*/true));
+  if (fuse_route_permute(L)) {
+    const PermuteArgs p = permute_args(d, L, ids, sc, counts, offsets, rows, inv, W, true);
+    const GatherArgs g = gather_args(d, L, x, rows, W + L.a_perm, W);
+    const bool fg = fuse_route_gather(d, L);
+    FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s, &p, fg ? &g : nullptr));
+    if (!fg) FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
+  } else {
+    FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
+    FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s,
+                          /*with_plan=*/true));
+  }
   FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s,
                         /*plan_done=*/true, /*fused_out=*/out, ids, inv));
   if (L.swap) return FMOE_OK;  // combined by combine_partials
@@ -578,8 +649,11 @@ int32_t fused_moe_launches_per_call(const fmoe_dims* dims) {
   if (check_dims(dims) != FMOE_OK) return -1;
   if (dims->T == 0) return 0;
   const Layout L = make_layout(*dims);
-  // router, permute (+plan), gather, gemm1, [finalize1], [quant_h], gemm2, combine
-  return 6 + (L.swap ? 1 : 0) + (L.fp8 ? 1 : 0);
+  // router [+ permute (+plan) [+ gather]], gemm1, [finalize1], [quant_h], gemm2, combine
+  int n = 4 + (L.fp8 ? 1 : 0) + (L.swap ? 1 : 0);
+  if (!fuse_route_permute(L)) n += 2;        // permute, gather
+  else if (!fuse_route_gather(*dims, L)) n += 1;  // gather
+  return n;
 }
 
 fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, const void* router_w,
@@ -619,6 +693,15 @@ fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, const void* 
   }
   *n_host = n;
   return FMOE_OK;
+}
+
+fmoe_status fused_moe_selftest_wait(void* ws, size_t ws_bytes, uint64_t budget_ns,
+                                    fmoe_stream stream) {
+  if (ws == nullptr) return FMOE_ERR_INVALID_ARG;
+  if (ws_bytes < sizeof(WsHeader)) return FMOE_ERR_WORKSPACE;
+  if (budget_ns > 10000000000ull) return FMOE_ERR_INVALID_ARG;  // at most 10 s
+  return cuda_status(launch_wait_selftest(static_cast<WsHeader*>(ws), budget_ns,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 fmoe_status fused_moe_get_device_status(const void* ws, fmoe_stream stream) {

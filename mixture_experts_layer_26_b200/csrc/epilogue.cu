@@ -1,9 +1,9 @@
 // Element-wise steps around the grouped GEMMs.
 //
-// finalize1: sum the split-K partials of the first contraction, apply the scale
-//   s1*sw13[e], h = SiLU(g)*u (gate = rows 0..I-1 of w13, up = rows I..2I-1), and keep a
-//   per-CTA max |h|.  FP8 format: h stays fp32 for the second quantisation.  bf16
-//   format: h is rounded to bf16 and is already the second GEMM's input.
+// finalize1: with split-K > 1, sum the first contraction's partials in split order,
+//   apply s1*sw13[e], h = SiLU(g)*u, keep a per-CTA max |h| (FP8: h stays fp32 for the
+//   second quantisation; bf16: h is rounded to bf16).  With split 1 the GEMM epilogue has
+//   already done this and the kernel returns at once.
 // quant_h: reduce the max |h| partials into the per-tensor scale s2 = amax/448 (or a
 //   static scale), then hq = e4m3(h * 448/amax) rounded to nearest even, saturating.
 // finalize2: sum the split-K partials of the second contraction, apply s2*sw2[e] and
@@ -276,6 +276,23 @@ __global__ void __launch_bounds__(kEwThreads) combine_kernel(CombineArgs a) {
   }
 }
 
+// Exercises the bounded mbarrier wait: thread 0 waits on a barrier that nothing
+// arrives at; the wait must give up after budget_ns and record ST_TIMEOUT.
+__global__ void wait_selftest_kernel(WsHeader* hdr, uint64_t budget_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool done = mbar_wait(&bar, 0, &abort_flag, &hdr->status, budget_ns);
+    hdr->pad0[0] = done ? 1 : 2;  // 2: the wait gave up, as it must
+  }
+}
+
 int ew_grid(size_t work_items, int num_sms) {
   const size_t per_cta = kEwThreads;
   size_t g = (work_items + per_cta - 1) / per_cta;
@@ -306,6 +323,11 @@ cudaError_t launch_finalize2(const Finalize2Args& a, int num_sms, cudaStream_t s
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
   return launch_k(combine_kernel, dim3(ew_grid(static_cast<size_t>(a.T) * a.H / 8, num_sms)),
                   dim3(kEwThreads), 0, s, a);
+}
+
+cudaError_t launch_wait_selftest(WsHeader* hdr, uint64_t budget_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(hdr, budget_ns);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_combine_partials(const CombinePartialsArgs& a, int num_sms, cudaStream_t s) {

@@ -29,7 +29,8 @@ struct alignas(256) WsHeader {
   int32_t split2;        // split-K factor of the second contraction (swap-AB only)
   int32_t amax_h_count;  // number of valid entries in amax_h_part
   int32_t router_ctas;   // number of valid entries in amax_x_part
-  int32_t pad0[10];
+  int32_t route_done;    // router tiles finished (fused permutation); zero between calls
+  int32_t pad0[9];
   float amax_x, s1, inv1;  // activation amax and the scale / inverse scale used for Aq
   float amax_h, s2, inv2;  // intermediate amax and the scale / inverse scale used for hq
   float pad1[10];

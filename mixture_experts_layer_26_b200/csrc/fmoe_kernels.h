@@ -45,26 +45,6 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-// ----------------------------------------------------------------------------- router
-struct RouterArgs {
-  const uint16_t* x;       // [T, H] bf16 bits
-  const uint16_t* wr;      // [E, H] bf16 bits
-  int32_t* topk_ids;       // [T, k]
-  float* topk_w;           // [T, k]
-  float* amax_part;        // [token tiles] per-tile max |x|
-  float* logits_g;         // [T, E] logits when the experts are split over CTAs
-  int32_t* tile_counters;  // [kRouterMaxTiles] zero between calls (self-resetting)
-  WsHeader* hdr;
-  int T, H, E, k;
-  int num_sms;
-  int experts_per_cta;     // set by the launcher
-};
-// Token tiles that may split their experts over several CTAs (counters in the header area).
-constexpr int kRouterMaxTiles = 4096;
-cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
-int router_tokens_per_cta(int T, int H, int E, int num_sms);
-int router_experts_per_warp(int E);
-
 // ----------------------------------------------------------------------------- permute
 // How the grouped GEMMs are planned from the per-expert offsets.
 struct PlanParams {
@@ -105,6 +85,36 @@ struct GatherArgs {
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
 
+// ----------------------------------------------------------------------------- router
+struct RouterArgs {
+  const uint16_t* x;       // [T, H] bf16 bits
+  const uint16_t* wr;      // [E, H] bf16 bits
+  int32_t* topk_ids;       // [T, k]
+  float* topk_w;           // [T, k]
+  float* amax_part;        // [token tiles] per-tile max |x|
+  float* logits_g;         // [T, E] logits when the experts are split over CTAs
+  int32_t* tile_counters;  // [kRouterMaxTiles] zero between calls (self-resetting)
+  WsHeader* hdr;
+  int T, H, E, k;
+  int num_sms;
+  int experts_per_cta;     // set by the launcher
+  // routing mode (fmoe_route_mode) and the grouped-sigmoid parameters
+  int mode, n_group, topk_group;
+  float routed_scaling;
+  const float* bias;       // [E] or null
+  // one-call path, small batches: the CTA that finishes the last token tile also runs
+  // the permutation (+ plan) and, if fuse_gather, the gather
+  int fuse_permute, fuse_gather;
+  int32_t* route_done;     // tiles finished so far (zero between calls)
+  PermuteArgs perm;
+  GatherArgs gather;
+};
+// Token tiles that may split their experts over several CTAs (counters in the header area).
+constexpr int kRouterMaxTiles = 4096;
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+int router_tokens_per_cta(int T, int H, int E, int num_sms);
+int router_experts_per_warp(int E);
+
 // ----------------------------------------------------------------------------- experts
 struct PlanArgs {
   const int32_t* offsets;  // [E + 1]
@@ -123,7 +133,7 @@ struct GemmArgs {
   int32_t* status;
   float* out;              // swap: partials [S][R][Nout]; normal: h [R, I] or y [R, H]
   uint16_t* out_bf16;      // first contraction, bf16 format: h rounded to bf16
-  float* h_out;            // swap-AB first contraction, FP8, split 1: h [R, I] fp32
+  float* h_out;            // swap-AB first contraction, FP8: h [R, I] fp32
   const float* w_scale;    // [E] per-expert weight scale (FP8) or null
   const float* topk_w;     // [R] flattened routing weights (normal, second contraction)
   const int32_t* sorted_rows;
@@ -192,6 +202,9 @@ struct CombinePartialsArgs {
   int fp8;
 };
 cudaError_t launch_combine_partials(const CombinePartialsArgs& a, int num_sms, cudaStream_t s);
+
+// A wait on an mbarrier nothing arrives at, bounded by budget_ns (records ST_TIMEOUT).
+cudaError_t launch_wait_selftest(WsHeader* hdr, uint64_t budget_ns, cudaStream_t s);
 
 struct CombineArgs {
   const float* y;           // [R, H]

@@ -47,15 +47,22 @@ constexpr int kThreads = 192;
 constexpr int kMaxStages = 12;
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 128-byte operand tile
 constexpr int kSwapBoxRows = 16;        // token rows per TMA box in the swap-AB variant
-constexpr int kAccCols = 256;           // TMEM columns per accumulator buffer
+// Accumulator buffers in the 512 TMEM columns: the normal variant's 256-column tiles
+// take two; the swap-AB variant's tiles are at most 64 columns (chunk_rows <= 64), so it
+// keeps eight, letting the epilogue (stores, split-K hand-off) lag up to seven tiles.
+constexpr int kMaxAccStages = 8;
+template <bool kSwap> struct AccLayout {
+  static constexpr int kStages = kSwap ? 8 : 2;
+  static constexpr int kCols = kSwap ? 64 : 256;
+};
 constexpr int kTmemCols = 512;
 constexpr int kSmemBudget = 220 * 1024;
 
 struct SmemCtl {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
+  uint64_t tmem_full[kMaxAccStages];
+  uint64_t tmem_empty[kMaxAccStages];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -65,7 +72,7 @@ struct SmemCtl {
 };
 
 struct Unit {
-  int e, row0, nrows, tile, s, kb0, kb1;
+  int e, c, row0, nrows, tile, s, kb0, kb1;
 };
 
 // Unit u -> (expert, chunk rows, output tile, split, K-block range).  The units of
@@ -84,6 +91,7 @@ __device__ __forceinline__ Unit decode_unit(long u, const Chunk* chunks, int per
   const int c = cq.cb + static_cast<int>(l2 % cq.nch);
   t.tile = static_cast<int>(l2 / cq.nch);
   const Chunk cc = chunks[c];
+  t.c = c;
   t.e = cc.e;
   t.row0 = cc.row0;
   t.nrows = cc.nrows;
@@ -111,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < AccLayout<kSwap>::kStages; ++i) {
       mbar_init(&ctl.tmem_full[i], 1);
       mbar_init(&ctl.tmem_empty[i], 4);
     }
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * AccLayout<kSwap>::kCols);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&ctl.full[stage], phase, abort_flag, a.status, budget)) {
             ok = false;
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
         if (!ok) break;
         tc_commit(&ctl.tmem_full[acc]);
-        if (++acc == 2) {
+        if (++acc == AccLayout<kSwap>::kStages) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -346,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const uint32_t tb =
-          tmem_base + static_cast<uint32_t>(acc * kAccCols) + (static_cast<uint32_t>(q * 32) << 16);
+          tmem_base + static_cast<uint32_t>(acc * AccLayout<kSwap>::kCols) + (static_cast<uint32_t>(q * 32) << 16);
       if constexpr (kSwap && kGemm == 1) {
         // lane r of quarter q: gate (r%32 < 16) or up (r%32 >= 16) of feature
         // tile*64 + 16q + r%16; column c = token row0 + c
@@ -375,8 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             }
           }
         } else {
+          // split-K: write this split's fp32 partial; finalize1 sums the splits in order
           const int feat = (lane & 16) ? a.I + f : f;
-          float* dst = a.out + (static_cast<size_t>(t.s) * a.R + t.row0) * a.Nout + feat;
+          const size_t plane = static_cast<size_t>(a.R) * a.Nout;
+          float* dst = a.out + static_cast<size_t>(t.s) * plane + static_cast<size_t>(t.row0) * a.Nout + feat;
           for (int c0 = 0; c0 < ncols; c0 += 16) {
             float v[16];
             tmem_ld16(tb + c0, v);
@@ -460,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.tmem_empty[acc]);
-      if (++acc == 2) {
+      if (++acc == AccLayout<kSwap>::kStages) {
         acc = 0;
         acc_phase ^= 1u;
       }

@@ -20,7 +20,7 @@
 // per token: k rounds of a shuffle argmax over (logit desc, expert index asc).
 #include <float.h>
 
-#include "fmoe_kernels.h"
+#include "permute_body.cuh"
 
 namespace fmoe {
 
@@ -42,6 +42,11 @@ __device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
   return av > bv || (av == bv && ae < be);
 }
 
+// Affinity of the grouped router: sigmoid evaluated in fp64, rounded once to fp32.
+__device__ __forceinline__ float sigmoid_f64(float l) {
+  return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(l))));
+}
+
 template <int TB, int EG>
 __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -49,6 +54,7 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
   float* logits = reinterpret_cast<float*>(smem + TB * a.H * 2);       // [TB][E]
   __shared__ float red[kRouterThreads / 32];
   __shared__ int is_last;
+  __shared__ int is_final;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, group = blockIdx.y;
@@ -161,9 +167,9 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
   if (split) {
     // The last of the gridDim.y CTAs of this token tile to finish picks the top-k
     // (counter reset for the next call by that CTA).
+    __threadfence();  // every writer orders its logits before the hand-off
     __syncthreads();
     if (threadIdx.x == 0) {
-      __threadfence();
       const int prev = atomicAdd(&a.tile_counters[tile], 1);
       is_last = prev == static_cast<int>(gridDim.y) - 1;
       if (is_last) {
@@ -181,6 +187,8 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
   __syncthreads();
 
   // ---- top-k, one warp per token
+  const bool grouped = a.mode == 1;
+  float* sbs = logits + TB * E;  // grouped: selection scores [TB][E]
   for (int t = warp; t < TB; t += kRouterThreads / 32) {
     const int tok = t0 + t;
     if (tok >= a.T) break;
@@ -190,10 +198,56 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int e = lane + 32 * j;
-      float l = e < E ? logits[t * E + e] : -INFINITY;
-      if (l != l) l = -INFINITY;  // NaN logits are unsupported; keep the selection well defined
+      float l = -INFINITY;
+      if (e < E) {
+        l = logits[t * E + e];
+        if (grouped) {
+          l = sigmoid_f64(l) + (a.bias != nullptr ? a.bias[e] : 0.f);
+          sbs[t * E + e] = l;
+        }
+      }
+      if (l != l) l = -INFINITY;  // NaN scores are unsupported; keep the selection well defined
       v[j] = l;
       taken[j] = e >= E;
+    }
+    if (grouped) {
+      // group score: the sum of the group's two largest selection scores
+      __syncwarp();
+      const int G = a.n_group, eg = E / a.n_group;
+      float gs = -INFINITY;
+      if (lane < G) {
+        float m1 = -INFINITY, m2 = -INFINITY;
+        for (int i = 0; i < eg; ++i) {
+          const float x = sbs[t * E + lane * eg + i];
+          if (x > m1) {
+            m2 = m1;
+            m1 = x;
+          } else if (x > m2) {
+            m2 = x;
+          }
+        }
+        gs = m1 + m2;
+      }
+      // keep the topk_group best groups (ties to the lower group)
+      uint32_t keep = 0;
+      bool gtaken = lane >= G;
+      for (int r = 0; r < a.topk_group; ++r) {
+        float bv = gtaken ? -INFINITY : gs;
+        int be = gtaken ? 0x7fffffff : lane;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+          if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
+        }
+        keep |= 1u << be;
+        if (lane == be) gtaken = true;
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && !((keep >> (e / eg)) & 1u)) v[j] = -INFINITY;
+      }
     }
     float top0 = 0.f, wsum = 0.f;
     float* wout = a.topk_w + static_cast<size_t>(tok) * a.k;
@@ -215,19 +269,54 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
 #pragma unroll
       for (int j = 0; j < kPer; ++j)
         if (lane + 32 * j == be) taken[j] = true;
-      if (r == 0) top0 = bv;
-      const float ex = expf(bv - top0);  // exp(l_j - l_max) of the j-th choice
-      wsum += ex;                         // summed in choice order
+      float ex;
+      if (grouped) {
+        ex = sigmoid_f64(logits[t * E + be]);  // the unbiased affinity of the j-th choice
+      } else {
+        if (r == 0) top0 = bv;
+        ex = expf(bv - top0);  // exp(l_j - l_max) of the j-th choice
+      }
+      wsum += ex;  // summed in choice order
       if (lane == 0) { iout[r] = be; wout[r] = ex; }
     }
-    if (lane == 0)
-      for (int r = 0; r < a.k; ++r) wout[r] = wout[r] / wsum;
+    if (lane == 0) {
+      const float scale = grouped ? a.routed_scaling : 1.f;
+      for (int r = 0; r < a.k; ++r) wout[r] = grouped ? wout[r] / wsum * scale : wout[r] / wsum;
+    }
+  }
+
+  if (a.fuse_permute) {
+    // The CTA that finishes the last token tile groups the rows by expert (and plans
+    // the GEMMs, and for small batches gathers the activations) for the whole batch.
+    __threadfence();  // this CTA's top-k results (and max |x|) before the hand-off
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int prev = atomicAdd(a.route_done, 1);
+      is_final = prev == static_cast<int>(gridDim.x) - 1;  // one top-k CTA per tile
+      if (is_final) {
+        *a.route_done = 0;
+        __threadfence();
+      }
+    }
+    __syncthreads();
+    if (!is_final) return;
+    int* ps = reinterpret_cast<int*>(smem);  // reuse: wc[8*E], cnt[E], base[E+1]
+    permute_body<kRouterThreads / 32>(a.perm, ps, ps + (kRouterThreads / 32) * E,
+                                      ps + (kRouterThreads / 32 + 1) * E);
+    if (a.fuse_gather) {
+      __syncthreads();
+      gather_rows(a.gather, warp, kRouterThreads / 32);
+    }
   }
 }
 
 template <int TB, int EG>
 cudaError_t launch_tb(RouterArgs a, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(TB) * a.H * 2 + static_cast<size_t>(TB) * a.E * 4;
+  size_t smem = static_cast<size_t>(TB) * a.H * 2 + static_cast<size_t>(TB) * a.E * 4 * (a.mode == 1 ? 2 : 1);
+  if (a.fuse_permute) {
+    const size_t need = static_cast<size_t>(kRouterThreads / 32 + 2) * a.E * 4 + 4;
+    smem = smem > need ? smem : need;
+  }
   cudaError_t err = set_max_dynamic_smem<router_kernel<TB, EG>>(160 * 1024);
   if (err != cudaSuccess) return err;
   // favour shared memory over L1 so that two CTAs fit per SM

@@ -43,6 +43,8 @@ class MoEShape:
     router_std: Optional[float] = None  # None: 1/sqrt(H)
     adversarial: bool = False
     name: str = ""
+    # group-limited sigmoid routing: (n_group, topk_group, routed_scaling); None = softmax
+    grouped: Optional[tuple] = None
 
     @property
     def R(self) -> int:
@@ -59,6 +61,13 @@ WORKLOADS = {
     "swapab_adversarial_fp8": dict(Ts=(8,), H=8192, I=8192, E=16, top_k=2, wdtype="fp8",
                                    adversarial=True),
     "prefill_fp8": dict(Ts=(4096,), H=4096, I=14336, E=8, top_k=2, wdtype="fp8"),
+    # the same Mixtral-like shapes with bf16 weights and activations
+    "mixtral_bf16_decode": dict(Ts=(1, 8, 32, 64), H=4096, I=14336, E=8, top_k=2, wdtype="bf16"),
+    "prefill_bf16": dict(Ts=(4096,), H=4096, I=14336, E=8, top_k=2, wdtype="bf16"),
+    # DeepSeek-V3-like shapes with its group-limited sigmoid router: 8 groups of 32
+    # experts, 4 groups kept, routed scaling 2.5, a seeded selection bias
+    "dsv3_grouped_fp8_decode": dict(Ts=(16, 64, 256), H=7168, I=2048, E=256, top_k=8,
+                                    wdtype="fp8", router_std=1.0, grouped=(8, 4, 2.5)),
 }
 
 
@@ -93,6 +102,7 @@ class MoEInputs:
     w2: torch.Tensor         # [E, H, I] uint8 (e4m3fn bits) or bf16
     w13_scale: Optional[torch.Tensor]  # [E] fp32 (FP8 formats only)
     w2_scale: Optional[torch.Tensor]   # [E] fp32
+    router_bias: Optional[torch.Tensor] = None  # [E] fp32 (grouped routing only)
 
 
 def make_activations(s: MoEShape, seed: int = 0, T: Optional[int] = None):
@@ -135,10 +145,17 @@ def make_weights(s: MoEShape, seed: int = 0):
     return w13, w2, (s13 if fp8 else None), (s2 if fp8 else None)
 
 
+def make_router_bias(s: MoEShape, seed: int = 0) -> Optional[torch.Tensor]:
+    """Selection bias of the grouped router: N(0, 0.02) per expert (None otherwise)."""
+    if s.grouped is None:
+        return None
+    return torch.randn(s.E, generator=_gen(seed, 5), dtype=torch.float32) * 0.02
+
+
 def make_inputs(s: MoEShape, seed: int = 0) -> MoEInputs:
     x, wr = make_activations(s, seed)
     w13, w2, s13, s2 = make_weights(s, seed)
-    return MoEInputs(s, x, wr, w13, w2, s13, s2)
+    return MoEInputs(s, x, wr, w13, w2, s13, s2, make_router_bias(s, seed))
 
 
 def bf16_bits(t: torch.Tensor):

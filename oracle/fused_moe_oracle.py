@@ -53,6 +53,9 @@ Readings where the pages are silent (each is listed in the design doc):
   R7 bf16 format: no quantisation; h is rounded to bf16 before the second
      contraction
   R8 the final sum is rounded fp64 -> fp32 -> bf16 (round to nearest even)
+The grouped sigmoid routing of router_grouped (a later variant of step 1-3 for the
+DeepSeek-V3-like shapes; the pages name DeepSeek-V3 but do not describe its router) is
+taken from DeepSeek-V3's published design; its readings D1-D5 are listed there.
 """
 from __future__ import annotations
 
@@ -173,6 +176,54 @@ def router(x_bits: np.ndarray, wr_bits: np.ndarray, top_k: int):
     sel = np.take_along_axis(p, ids, axis=1)
     w = sel / sel.sum(axis=1, keepdims=True)           # renormalised over the top-k
     return ids, w.astype(np.float32), logits
+
+
+def sigmoid_scores(logits: np.ndarray) -> np.ndarray:
+    """Affinities of the grouped routing: sigmoid of the fp32 logits, evaluated in fp64
+    and rounded once to fp32 (reading D1)."""
+    l64 = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    return (1.0 / (1.0 + np.exp(-l64))).astype(np.float32)
+
+
+def router_grouped(x_bits: np.ndarray, wr_bits: np.ndarray, top_k: int, n_group: int,
+                   topk_group: int, bias=None, routed_scaling: float = 1.0):
+    """Group-limited sigmoid routing (the DeepSeek-V3 router; readings D1-D5).
+
+    D1 s = fp32(sigmoid(logit)) with the logits of router_logits (canonical order);
+    D2 selection scores sb = s + bias[e], one fp32 addition (bias 0 when absent);
+    D3 the E experts form n_group groups of E/n_group consecutive experts; a group's
+       score is the sum (fp32) of its two largest sb; the topk_group best groups are
+       kept, ties to the lower group index;
+    D4 top-k experts by sb among the kept groups, descending, ties to the lower index;
+    D5 weights: the unbiased s of the chosen experts over their sum (fp64), times
+       routed_scaling, stored as fp32.
+    Returns topk_ids [T,k] int32, topk_w [T,k] float32, s [T,E], sb [T,E] float32."""
+    logits = router_logits(x_bits, wr_bits)
+    ids, w, s, sb = grouped_select(logits, top_k, n_group, topk_group, bias, routed_scaling)
+    return ids, w, s, sb
+
+
+def grouped_select(logits, top_k, n_group, topk_group, bias=None, routed_scaling=1.0):
+    """Steps D1-D5 of router_grouped on given fp32 logits [T, E]."""
+    logits = np.asarray(logits, np.float32)
+    T, E = logits.shape
+    eg = E // n_group
+    assert E % n_group == 0 and eg >= 2 and topk_group * eg >= top_k
+    s = sigmoid_scores(logits)
+    b = np.zeros(E, np.float32) if bias is None else np.asarray(bias, np.float32)
+    sb = (s + b[None, :]).astype(np.float32)
+    grp = np.sort(sb.reshape(T, n_group, eg), axis=-1)            # ascending
+    gscore = (grp[..., -1] + grp[..., -2]).astype(np.float32)      # two largest
+    gidx = np.broadcast_to(np.arange(n_group), (T, n_group))
+    keep_g = np.lexsort((gidx, -gscore), axis=-1)[:, :topk_group]
+    keep = np.zeros((T, n_group), bool)
+    np.put_along_axis(keep, keep_g, True, axis=1)
+    masked = np.where(np.repeat(keep, eg, axis=1), sb, -np.inf).astype(np.float32)
+    eidx = np.broadcast_to(np.arange(E), (T, E))
+    ids = np.lexsort((eidx, -masked), axis=-1)[:, :top_k].astype(np.int32)
+    sel = np.take_along_axis(s, ids, axis=1).astype(np.float64)
+    w = sel / sel.sum(axis=1, keepdims=True) * float(np.float32(routed_scaling))
+    return ids, w.astype(np.float32), s, sb
 
 
 # --------------------------------------------------------------------------------------
@@ -307,15 +358,19 @@ def combine(y, inv_perm, T, top_k):
 
 
 def fused_moe(x_bits, wr_bits, w13, w2, top_k, fp8=True, w13_scale=None, w2_scale=None,
-              a1_scale=0.0, a2_scale=0.0):
+              a1_scale=0.0, a2_scale=0.0, grouped=None):
     """The whole layer on host arrays.  x_bits [T,H] / wr_bits [E,H] are bf16 bit
     patterns (uint16); w13 [E,2I,H], w2 [E,H,I] are e4m3 codes (uint8) or bf16 bits.
+    grouped: None for softmax top-k routing, else the router_grouped parameters.
     Returns a dict with every intermediate the GPU path also exposes."""
     x_bits = np.asarray(x_bits)
     T, H = x_bits.shape
     E = wr_bits.shape[0]
     I = w2.shape[2]
-    ids, w, logits = router(x_bits, wr_bits, top_k)
+    if grouped is None:
+        ids, w, logits = router(x_bits, wr_bits, top_k)
+    else:   # dict(n_group=, topk_group=, bias=, routed_scaling=)
+        ids, w, logits, _ = router_grouped(x_bits, wr_bits, top_k, **grouped)
     counts, offsets, sorted_rows, inv_perm = permute(ids, E)
     a_perm, s1, inv1, amax_x = permute_quant(x_bits, sorted_rows, top_k, fp8, a1_scale)
     y, h, hq, s2 = experts(a_perm, offsets, sorted_rows, w, w13, w2, H, I, E, fp8, s1,

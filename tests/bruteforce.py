@@ -112,3 +112,27 @@ def brute_force(x_bits, wr_bits, w13, w2, top_k, fp8, w13_scale=None, w2_scale=N
                 acc[mcol] += weights[t][j] * yv
         out.append([_bf16(_f32(v)) for v in acc])
     return dict(ids=ids, weights=weights, logits=logits, out=out, h=hs)
+
+
+def grouped_routing(logits, top_k, n_group, topk_group, bias=None, routed_scaling=1.0):
+    """Group-limited sigmoid routing token by token with Python floats, from given
+    fp32 logits (their summation order is pinned separately)."""
+    ex = [[float(v) for v in row] for row in logits]
+    T, E = len(ex), len(ex[0])
+    eg = E // n_group
+    b = [0.0] * E if bias is None else [float(v) for v in bias]
+    ids, ws = [], []
+    for t in range(T):
+        s = [_f32(1.0 / (1.0 + math.exp(-_f32(l)))) for l in ex[t]]
+        sb = [_f32(s[e] + b[e]) for e in range(E)]
+        gs = []
+        for g in range(n_group):
+            members = sorted(sb[g * eg:(g + 1) * eg], reverse=True)
+            gs.append(_f32(members[0] + members[1]))
+        kept = sorted(range(n_group), key=lambda g: (-gs[g], g))[:topk_group]
+        cand = [e for e in range(E) if e // eg in kept]
+        chosen = sorted(cand, key=lambda e: (-sb[e], e))[:top_k]
+        tot = math.fsum(s[e] for e in chosen)
+        ids.append(chosen)
+        ws.append([_f32(s[e] / tot * _f32(routed_scaling)) for e in chosen])
+    return ids, ws

@@ -25,11 +25,21 @@ def np_inputs(inp: "minp.MoEInputs") -> dict:
     )
 
 
+def grouped_args(inp):
+    """The oracle's grouped-routing parameters of these inputs (None for softmax)."""
+    if inp.shape.grouped is None:
+        return None
+    n_group, topk_group, scaling = inp.shape.grouped
+    return dict(n_group=n_group, topk_group=topk_group, routed_scaling=scaling,
+                bias=inp.router_bias.numpy())
+
+
 def run_oracle(oracle_mod, inp, a1_scale=0.0, a2_scale=0.0):
     d = np_inputs(inp)
     return oracle_mod.fused_moe(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], d["top_k"],
                                 fp8=d["fp8"], w13_scale=d["w13_scale"],
-                                w2_scale=d["w2_scale"], a1_scale=a1_scale, a2_scale=a2_scale)
+                                w2_scale=d["w2_scale"], a1_scale=a1_scale, a2_scale=a2_scale,
+                                grouped=grouped_args(inp))
 
 
 def bf16_bits_to_float(bits) -> np.ndarray:

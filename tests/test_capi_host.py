@@ -23,7 +23,7 @@ def header_symbols():
 
 def test_header_symbols_are_exported():
     syms = header_symbols()
-    assert len(syms) == 15
+    assert len(syms) == 16
     assert set(syms) == set(capi.EXPORTED)
     lib = ctypes.CDLL(capi.LIB_PATH)
     for s in syms:
@@ -31,7 +31,7 @@ def test_header_symbols_are_exported():
 
 
 def test_abi_version_and_strings():
-    assert capi.abi_version() == 1
+    assert capi.abi_version() == 2
     for code, name in [(0, "FMOE_OK"), (1, "FMOE_ERR_INVALID_ARG"), (2, "FMOE_ERR_UNSUPPORTED"),
                        (3, "FMOE_ERR_WORKSPACE"), (4, "FMOE_ERR_CUDA"), (5, "FMOE_ERR_TIMEOUT"),
                        (6, "FMOE_ERR_DEVICE_BOUNDS")]:
@@ -111,15 +111,17 @@ def test_validation_codes_without_cuda():
 
 
 def test_launch_counts():
-    assert capi.fused_moe_launches_per_call(dims(T=4, variant="swap_ab")) == 8
-    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal")) == 7
-    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="swap_ab")) == 7
-    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="normal")) == 6
+    # small batch: router (+ permute, plan, gather), gemm1, finalize1 (swap-AB),
+    # quant_h (FP8), gemm2, combine
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="swap_ab")) == 6
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal")) == 5
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="swap_ab")) == 5
     assert capi.fused_moe_launches_per_call(dims(T=0)) == 0
     assert capi.fused_moe_launches_per_call(dims(k=9)) == -1
-    # AUTO: swap-AB while an expert averages at most 64 rows
-    assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 8
-    assert capi.fused_moe_launches_per_call(dims(T=257, E=8, k=2)) == 7
+    # gathered rows above 128 KB: the gather is its own launch
+    assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 7
+    # more than 2048 routed rows: permute and gather are their own launches (normal variant)
+    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2)) == 7
 
 
 def test_zero_tokens_is_a_noop():
@@ -147,3 +149,21 @@ def test_step_validation():
                                   check=False) == capi.FMOE_ERR_INVALID_ARG    # FP8, no scales
     assert capi.fused_moe_combine(d, _T(FAKE), _T(0), _T(FAKE), stream=0,
                                   check=False) == capi.FMOE_ERR_INVALID_ARG
+
+
+def test_routing_descriptor_validation():
+    def grouped(n_group, topk_group, scaling=2.5, bias=None, k=8, E=64):
+        r = capi.FmoeRouting(capi.FMOE_ROUTE_SIGMOID_GROUPED, n_group, topk_group, scaling, bias)
+        return call_fused(capi.make_dims(4, 256, 512, E, k, True, routing=r))
+    assert grouped(8, 4) == capi.FMOE_ERR_WORKSPACE          # valid: stops at the ws check
+    assert grouped(8, 1) == capi.FMOE_ERR_WORKSPACE          # 1 group of 8 experts, k = 8: valid
+    assert grouped(16, 1, k=8) == capi.FMOE_ERR_INVALID_ARG  # 1 group of 4 experts < k
+    assert grouped(7, 2) == capi.FMOE_ERR_INVALID_ARG        # E % n_group != 0
+    assert grouped(64, 8, k=2) == capi.FMOE_ERR_INVALID_ARG  # groups of 1 expert
+    assert grouped(8, 9) == capi.FMOE_ERR_INVALID_ARG        # topk_group > n_group
+    assert grouped(8, 4, scaling=0.0) == capi.FMOE_ERR_INVALID_ARG
+    assert grouped(8, 4, bias=FAKE + 2) == capi.FMOE_ERR_UNSUPPORTED   # misaligned bias
+    bad = capi.FmoeRouting(7, 1, 1, 1.0, None)
+    assert call_fused(capi.make_dims(4, 256, 512, 8, 2, True, routing=bad)) == capi.FMOE_ERR_INVALID_ARG
+    softmax = capi.FmoeRouting(capi.FMOE_ROUTE_SOFTMAX, 0, 0, 0.0, None)
+    assert call_fused(capi.make_dims(4, 256, 512, 8, 2, True, routing=softmax)) == capi.FMOE_ERR_WORKSPACE

@@ -20,7 +20,7 @@ import torch
 
 from oracle import fused_moe_oracle as O
 from mixture_experts_layer_26_b200 import inputs as minp
-from bruteforce import brute_force, exact_logits
+from bruteforce import brute_force, exact_logits, grouped_routing as brute_grouped
 from helpers import np_inputs, run_oracle, max_rel_err, tiny_shape, bf16_bits_to_float, torch_bf16_bits
 
 
@@ -386,3 +386,79 @@ def test_tiny_bf16_regression_golden():
     assert r["counts"].tolist() == doc["counts"]
     assert r["sorted_rows"].tolist() == doc["sorted_rows"]
     assert r["out"].astype(int).tolist() == doc["out_bf16_bits"]
+
+
+# ----------------------------------------------------------------------------- grouped routing
+
+def _sig(v):
+    return 1.0 / (1.0 + math.exp(-v))
+
+
+def _onehot_router(table):
+    """x = e_t, router_w[:, t] = table[t]: logit[t, e] = table[t][e] exactly."""
+    table = np.asarray(table, np.float32)
+    T, E = table.shape
+    H = 256
+    x = np.zeros((T, H), np.float32)
+    x[np.arange(T), np.arange(T)] = 1.0
+    wr = np.zeros((E, H), np.float32)
+    wr[:, :T] = table.T
+    return _bits(x), _bits(wr)
+
+
+def test_grouped_routing_closed_form():
+    # 8 experts in 4 groups of 2, keep 2 groups, pick 2 experts.
+    # token 0: expert 7 has the largest score but its group {6, 7} scores s(-1)+s(5)
+    # = 1.262, below {0, 1}: s(4)+s(3) = 1.935 and {4, 5}: 2 s(2) = 1.762, so the
+    # choice is experts 0 then 1.  token 1: all equal -> groups 0, 1 -> experts 0, 1.
+    table = [[4, 3, 0, 0, 2, 2, -1, 5],
+             [1, 1, 1, 1, 1, 1, 1, 1]]
+    xb, wb = _onehot_router(table)
+    ids, w, s, sb = O.router_grouped(xb, wb, 2, n_group=4, topk_group=2, routed_scaling=2.5)
+    assert ids.tolist() == [[0, 1], [0, 1]]
+    ref0 = [_sig(4) / (_sig(4) + _sig(3)) * 2.5, _sig(3) / (_sig(4) + _sig(3)) * 2.5]
+    assert np.allclose(w[0], ref0, rtol=1e-6, atol=0)
+    assert np.allclose(w[1], [1.25, 1.25], rtol=1e-7, atol=0)
+    # a bias of +1 on expert 7 lifts group {6, 7} to s(-1) + s(5) + 1 = 2.262: the kept
+    # groups become {6, 7} and {0, 1}; by biased score expert 7 then expert 0, and the
+    # weights use the unbiased scores
+    bias = np.zeros(8, np.float32)
+    bias[7] = 1.0
+    ids, w, _, sb = O.router_grouped(xb, wb, 2, n_group=4, topk_group=2, bias=bias)
+    assert ids[0].tolist() == [7, 0]
+    assert np.allclose(w[0], [_sig(5) / (_sig(5) + _sig(4)), _sig(4) / (_sig(5) + _sig(4))],
+                       rtol=1e-6, atol=0)
+    assert sb[0, 7] == np.float32(np.float32(_sig(5)) + np.float32(1.0))
+
+
+def test_grouped_sigmoid_is_fp64_rounded_once():
+    l = np.array([[-3.5, 0.0, 0.1234567, 7.25, -20.0, 40.0]], np.float32)
+    got = O.sigmoid_scores(l)
+    ref = np.array([[_sig(float(v)) for v in l[0]]], np.float64).astype(np.float32)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("seed,T,E,G,M,k", [(0, 12, 16, 4, 2, 4), (1, 9, 32, 8, 3, 6),
+                                            (2, 5, 64, 8, 4, 8)])
+def test_grouped_routing_matches_bruteforce(seed, T, E, G, M, k):
+    s_ = tiny_shape(T, 256, 128, E, k, "fp8", router_std=0.5)
+    x, wr = minp.make_activations(s_, seed=seed)
+    xb, wb = minp.bf16_bits(x), minp.bf16_bits(wr)
+    rng = np.random.default_rng(seed)
+    bias = (rng.standard_normal(E) * 0.05).astype(np.float32)
+    ids, w, s, sb = O.router_grouped(xb, wb, k, n_group=G, topk_group=M, bias=bias,
+                                     routed_scaling=2.5)
+    # the brute force starts from the same fp32 logits (pinned by the canonical-order
+    # tests) and redoes the sigmoid, grouping, selection and weights on its own
+    logits = O.router_logits(xb, wb)
+    bids, bw = brute_grouped(logits, k, G, M, bias, 2.5)
+    assert ids.tolist() == bids
+    assert np.allclose(w, np.array(bw), rtol=1e-6, atol=0)
+    eg = E // G
+    for t in range(T):
+        assert np.isclose(float(w[t].astype(np.float64).sum()), 2.5, rtol=1e-6)
+        assert len(set(ids[t].tolist())) == k
+        groups = sb[t].reshape(G, eg)
+        gscore = np.sort(groups, axis=1)[:, -1] + np.sort(groups, axis=1)[:, -2]
+        kept = set(sorted(range(G), key=lambda g: (-gscore[g], g))[:M])
+        assert {int(e) // eg for e in ids[t]} <= kept
