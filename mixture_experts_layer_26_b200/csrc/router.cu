@@ -96,7 +96,9 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
   const int steps = H / 256;  // chunks per lane
   const int e_begin = group * a.experts_per_cta;
   const int e_end = min(E, e_begin + a.experts_per_cta);
-  constexpr int U = 2;  // chunk steps whose router rows are loaded together
+  // chunk steps whose router rows are loaded together: more when a warp owns fewer
+  // experts, so that every warp keeps about eight 16-byte loads in flight
+  constexpr int U = EG >= 4 ? 2 : 8 / EG;
   // Accumulators acc[t][g] are updated in pairs with one paired FMA (each component
   // rounds exactly like a scalar fmaf), element by element in ascending order, so
   // every logit keeps the canonical summation order.
