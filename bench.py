@@ -51,8 +51,11 @@ from mixture_experts_layer_26_b200 import inputs as minp  # noqa: E402
 METRIC = "fused-MoE tokens/s; achieved HBM GB/s (decode) / FP8 TFLOPS (prefill) vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 2 ** 20
+# sources whose hash an ncu summary of a GEMM kernel records (pair kernels: gemm_pair.cu)
 GEMM_SOURCES = ("mixture_experts_layer_26_b200/csrc/gemm.cu",
                 "mixture_experts_layer_26_b200/csrc/fmoe_common.cuh")
+PAIR_GEMM_SOURCES = ("mixture_experts_layer_26_b200/csrc/gemm_pair.cu",
+                     "mixture_experts_layer_26_b200/csrc/fmoe_common.cuh")
 
 
 # --------------------------------------------------------------------------- helpers
@@ -66,9 +69,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def gemm_source_hash() -> str:
+def gemm_source_hash(kernel: str = "") -> str:
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
+    for rel in (PAIR_GEMM_SOURCES if "pair" in kernel else GEMM_SOURCES):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -87,7 +90,7 @@ def profiled_traffic(kernel: str, workload_tag: str):
         text = open(os.path.join(pdir, name)).read()
         t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
         hsh = re.search(r"source_hash:\s*([0-9a-f]+)", text)
-        if t and hsh and hsh.group(1) == gemm_source_hash():
+        if t and hsh and hsh.group(1) == gemm_source_hash(kernel):
             return float(t.group(1))
     return None
 
@@ -373,7 +376,8 @@ def run_ours(args, rank, world, local_rank):
     esz = 1 if fp8 else 2
     peaks, peak_kind = load_peaks()
     dom = max(kern_ms, key=kern_ms.get)
-    variant = "swap_ab" if "swapab" in "".join(kern_ms) else "normal"
+    names = "".join(kern_ms)
+    variant = "swap_ab" if "swapab" in names else ("normal_pair" if "pair" in names else "normal")
     gemm1_bytes = touched * 2 * s.H * s.I * esz          # weights of the touched experts
     gemm2_bytes = touched * s.H * s.I * esz
     gemm1_flops = 4.0 * s.R * s.H * s.I                  # gate and up: 2 x (2 R H I)
@@ -445,7 +449,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_fp8_decode", choices=sorted(minp.WORKLOADS))
     ap.add_argument("--T", type=int, default=64)
-    ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal", "normal_pair"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -88,11 +88,19 @@ typedef enum {
 } fmoe_wdtype;
 
 /* Tile shape of the grouped GEMMs.  AUTO picks SWAP_AB when an expert receives at
- * most 64 rows on average (T*k/E <= 64) and NORMAL otherwise.  SWAP_AB puts 128 weight
- * rows in the MMA's M slot and the expert's tokens in N (decode); NORMAL puts 128
- * tokens in M and 256 weight rows in N (prefill).  Both give the same results up to
- * fp32 summation order. */
-typedef enum { FMOE_VARIANT_AUTO = 0, FMOE_VARIANT_SWAP_AB = 1, FMOE_VARIANT_NORMAL = 2 } fmoe_variant;
+ * most 64 rows on average (T*k/E <= 64), NORMAL for 65..128 rows and NORMAL_PAIR above.
+ * SWAP_AB puts 128 weight rows in the MMA's M slot and the expert's tokens in N
+ * (decode); NORMAL puts 128 tokens in M and 256 weight rows in N (prefill); NORMAL_PAIR
+ * runs the NORMAL tiles on pairs of CTAs (clusters of two on one TPC) that share one
+ * MMA over 256 tokens x 256 weight rows, each CTA staging half of the weight rows.
+ * NORMAL and NORMAL_PAIR give identical results; SWAP_AB agrees with them up to fp32
+ * summation order. */
+typedef enum {
+  FMOE_VARIANT_AUTO = 0,
+  FMOE_VARIANT_SWAP_AB = 1,
+  FMOE_VARIANT_NORMAL = 2,
+  FMOE_VARIANT_NORMAL_PAIR = 3
+} fmoe_variant;
 
 /* How tokens choose experts.
  *  FMOE_ROUTE_SOFTMAX: the k largest logits; weights = softmax over all E experts

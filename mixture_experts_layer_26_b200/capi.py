@@ -29,7 +29,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 FMOE_OK, FMOE_ERR_INVALID_ARG, FMOE_ERR_UNSUPPORTED, FMOE_ERR_WORKSPACE = 0, 1, 2, 3
 FMOE_ERR_CUDA, FMOE_ERR_TIMEOUT, FMOE_ERR_DEVICE_BOUNDS = 4, 5, 6
 FMOE_BF16, FMOE_FP8_E4M3 = 0, 1
-VARIANTS = {"auto": 0, "swap_ab": 1, "normal": 2}
+VARIANTS = {"auto": 0, "swap_ab": 1, "normal": 2, "normal_pair": 3}
 
 EXPORTED = (
     "fused_moe_abi_version", "fused_moe_status_string", "fused_moe_workspace_size",

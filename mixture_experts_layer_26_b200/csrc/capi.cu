@@ -27,7 +27,7 @@ constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // bounded mbarrier waits: 2 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-  bool fp8 = false, swap = false;
+  bool fp8 = false, swap = false, pair = false;
   int R = 0, chunk_rows = 0, max_chunks = 0, s1max = 0, s2max = 0;
   size_t hdr = 0, counters = 0, amax_x = 0, amax_h = 0, chunks = 0, logits = 0;
   size_t ids = 0, tw = 0, counts = 0, offsets = 0, rows = 0, inv = 0;
@@ -41,7 +41,7 @@ fmoe_status check_dims(const fmoe_dims* d) {
       d->top_k > d->E)
     return FMOE_ERR_INVALID_ARG;
   if (d->wdtype != FMOE_BF16 && d->wdtype != FMOE_FP8_E4M3) return FMOE_ERR_INVALID_ARG;
-  if (d->variant < FMOE_VARIANT_AUTO || d->variant > FMOE_VARIANT_NORMAL)
+  if (d->variant < FMOE_VARIANT_AUTO || d->variant > FMOE_VARIANT_NORMAL_PAIR)
     return FMOE_ERR_INVALID_ARG;
   if (d->routing != nullptr) {
     const fmoe_routing& r = *d->routing;
@@ -74,11 +74,15 @@ Layout make_layout(const fmoe_dims& d) {
   const int R = T * d.top_k;
   L.R = R;
   int variant = d.variant;
-  if (variant == FMOE_VARIANT_AUTO)
-    variant = ((R + E - 1) / E <= 64) ? FMOE_VARIANT_SWAP_AB : FMOE_VARIANT_NORMAL;
+  if (variant == FMOE_VARIANT_AUTO) {
+    const int avg = (R + E - 1) / E;
+    variant = avg <= 64 ? FMOE_VARIANT_SWAP_AB : avg <= 128 ? FMOE_VARIANT_NORMAL : FMOE_VARIANT_NORMAL_PAIR;
+  }
   L.swap = variant == FMOE_VARIANT_SWAP_AB;
+  L.pair = variant == FMOE_VARIANT_NORMAL_PAIR;
   // an expert receives at most T rows (one per token)
-  L.chunk_rows = L.swap ? std::min(64, static_cast<int>(align_up(std::max(T, 1), 16))) : 128;
+  L.chunk_rows = L.swap ? std::min(64, static_cast<int>(align_up(std::max(T, 1), 16)))
+                        : (L.pair ? 256 : 128);
   L.max_chunks = R / L.chunk_rows + std::min(E, R) + 1;
   const size_t es = L.fp8 ? 1 : 2;
   const size_t p1_plane = static_cast<size_t>(R) * 2 * I * 4;
@@ -411,7 +415,10 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g.chunk_rows = L.chunk_rows;
   g.nstages = gemm_stages(swap, L.chunk_rows);
   g.wait_budget_ns = kWaitBudgetNs;
-  FMOE_LAUNCH(swap ? "gemm1_swapab" : "gemm1_normal", launch_gemm(g, fp8, swap, 1, sms, s), s);
+  if (L.pair)
+    FMOE_LAUNCH("gemm1_pair", launch_gemm_pair(g, fp8, 1, sms, s), s);
+  else
+    FMOE_LAUNCH(swap ? "gemm1_swapab" : "gemm1_normal", launch_gemm(g, fp8, swap, 1, sms, s), s);
 
   if (swap) {
     // split-K > 1: finish h from the partials (returns at once when the plan chose split 1)
@@ -453,7 +460,10 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g2.K = I;
   g2.Nout = H;
   g2.rows_per_expert = H;
-  FMOE_LAUNCH(swap ? "gemm2_swapab" : "gemm2_normal", launch_gemm(g2, fp8, swap, 2, sms, s), s);
+  if (L.pair)
+    FMOE_LAUNCH("gemm2_pair", launch_gemm_pair(g2, fp8, 2, sms, s), s);
+  else
+    FMOE_LAUNCH(swap ? "gemm2_swapab" : "gemm2_normal", launch_gemm(g2, fp8, swap, 2, sms, s), s);
 
   if (swap && fused_out != nullptr) {
     CombinePartialsArgs c{};

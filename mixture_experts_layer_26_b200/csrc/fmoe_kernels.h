@@ -149,6 +149,9 @@ struct GemmArgs {
 cudaError_t launch_gemm(const GemmArgs& a, bool fp8, bool swap_ab, int gemm, int num_sms,
                         cudaStream_t s);
 int gemm_stages(bool swap_ab, int chunk_rows);
+// The normal variant on CTA pairs (chunks of up to 256 rows); same arguments and outputs
+// as launch_gemm(..., swap_ab = false, ...).
+cudaError_t launch_gemm_pair(const GemmArgs& a, bool fp8, int gemm, int num_sms, cudaStream_t s);
 
 struct Finalize1Args {
   const float* part;        // [S][R][2I]

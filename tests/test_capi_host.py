@@ -122,6 +122,23 @@ def test_launch_counts():
     assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 7
     # more than 2048 routed rows: permute and gather are their own launches (normal variant)
     assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2)) == 7
+    # the CTA-pair kernels launch once per contraction like the one-CTA ones
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal_pair")) == 5
+    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2, variant="normal_pair")) == 7
+
+
+def test_variant_choice_and_pair_workspace():
+    # AUTO: <= 64 rows per expert on average -> swap-AB; 65..128 -> normal; above -> pairs.
+    # Pair chunks hold 256 rows, so the workspace never grows over the one-CTA normal one,
+    # and a forced variant outside AUTO's choice is still accepted.
+    ws = capi.workspace_size
+    assert ws(dims(T=4096, H=4096, I=1024, variant="normal_pair")) <= \
+        ws(dims(T=4096, H=4096, I=1024, variant="normal"))
+    for v in ("auto", "swap_ab", "normal", "normal_pair"):
+        assert ws(dims(T=300, variant=v)) > 0
+    bad = dims()
+    bad.variant = 4
+    assert call_fused(bad) == capi.FMOE_ERR_INVALID_ARG
 
 
 def test_zero_tokens_is_a_noop():

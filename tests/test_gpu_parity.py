@@ -130,6 +130,9 @@ SMALL = [
     ("fp8_dsv3_gate", (64, 512, 256, 64, 8, "fp8"), {"router_std": 1.0}),
     ("fp8_grouped", (64, 512, 256, 64, 8, "fp8"), {"router_std": 1.0, "grouped": (8, 4, 2.5)}),
     ("bf16_grouped_small_groups", (24, 256, 256, 32, 4, "bf16"), {"grouped": (16, 3, 1.0)}),
+    # more than 256 rows per expert: several CTA-pair chunks with ragged tails
+    ("fp8_pair_chunks", (700, 512, 384, 2, 1, "fp8"), {}),
+    ("bf16_pair_chunks", (600, 256, 256, 3, 2, "bf16"), {}),
 ]
 
 
@@ -146,7 +149,7 @@ def small_cases():
     return get
 
 
-@pytest.mark.parametrize("variant", ["swap_ab", "normal"])
+@pytest.mark.parametrize("variant", ["swap_ab", "normal", "normal_pair"])
 @pytest.mark.parametrize("name", [c[0] for c in SMALL])
 def test_small_steps_match_oracle(small_cases, name, variant):
     inp, g, ref = small_cases(name)
@@ -177,6 +180,17 @@ def test_small_fused_equals_steps_and_variants_agree(small_cases, name):
     # deterministic: a second call gives the same bits
     out_a2, _ = run_fused(inp, g, "auto")
     assert np.array_equal(out_a, out_a2)
+
+
+@pytest.mark.parametrize("name", ["tiny_bf16", "fp8_ragged", "fp8_multichunk", "fp8_pair_chunks",
+                                  "bf16_pair_chunks", "fp8_many_experts"])
+def test_pair_variant_equals_normal(small_cases, name):
+    """The CTA-pair kernel runs the normal variant's tiles with the same K order and the
+    same epilogue arithmetic: identical output bits."""
+    inp, g, _ = small_cases(name)
+    out_n, _ = run_fused(inp, g, "normal")
+    out_p, _ = run_fused(inp, g, "normal_pair")
+    assert np.array_equal(out_n, out_p)
 
 
 def test_static_scales(small_cases):
@@ -269,6 +283,10 @@ def test_full_size_matches_oracle(full_weights, workload, T):
         other = "normal" if (s.R + s.E - 1) // s.E <= 64 else "swap_ab"
         out_o, _ = run_fused(inp, g, other)
         assert max_rel_err(bf16_bits_to_float(out_o), ref["out64"]) <= TOL[s.wdtype]
+    if workload.startswith("prefill"):
+        # AUTO runs the CTA-pair kernel here; the one-CTA normal kernel gives the same bits
+        out_n, _ = run_fused(inp, g, "normal")
+        assert np.array_equal(out_n, out_f)
 
 
 ROUTER_SHAPES = [("mixtral_fp8_decode", T) for T in (1, 64)] + \
@@ -313,7 +331,9 @@ def test_router_full_shapes(workload, T):
 
 
 @pytest.mark.parametrize("name,variant", [("fp8_ragged", "swap_ab"), ("fp8_multichunk", "normal"),
-                                          ("bf16_multichunk", "swap_ab")])
+                                          ("bf16_multichunk", "swap_ab"),
+                                          ("fp8_pair_chunks", "normal_pair"),
+                                          ("bf16_pair_chunks", "normal_pair")])
 def test_poisoned_workspace_and_outputs_are_fully_rewritten(small_cases, name, variant):
     """Workspace (apart from its initialised header) and every output start as NaN
     bytes: a kernel that read a region it had not written, or left an output element
