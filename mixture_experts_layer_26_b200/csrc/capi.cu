@@ -368,7 +368,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
                          const void* w13, const void* w2, const fmoe_scales* sc, float* y,
                          char* W, cudaStream_t s, bool plan_done = false,
                          void* fused_out = nullptr, const int32_t* ids = nullptr,
-                         const int32_t* inv = nullptr) {
+                         const int32_t* inv = nullptr, bool plan_two_back = false) {
   const int sms = num_sms();
   const bool fp8 = L.fp8, swap = L.swap;
   const int H = d.H, I = d.I, E = d.E, R = L.R;
@@ -414,6 +414,9 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g.rows_per_expert = 2 * I;
   g.chunk_rows = L.chunk_rows;
   g.nstages = gemm_stages(swap, L.chunk_rows);
+  // the first contraction may prefetch weights when its plan came two launches back (the
+  // gather ran in between); the second one always may (gemm1 at least sits in between)
+  g.prefetch_w = plan_two_back ? 1 : 0;
   g.wait_budget_ns = kWaitBudgetNs;
   if (L.pair)
     FMOE_LAUNCH("gemm1_pair", launch_gemm_pair(g, fp8, 1, sms, s), s);
@@ -460,6 +463,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g2.K = I;
   g2.Nout = H;
   g2.rows_per_expert = H;
+  g2.prefetch_w = 1;
   if (L.pair)
     FMOE_LAUNCH("gemm2_pair", launch_gemm_pair(g2, fp8, 2, sms, s), s);
   else
@@ -522,19 +526,21 @@ fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   int32_t* rows = reinterpret_cast<int32_t*>(W + L.rows);
   int32_t* inv = reinterpret_cast<int32_t*>(W + L.inv);
   float* y = reinterpret_cast<float*>(W + L.y);
+  bool plan_two_back = true;  // the plan-writing launch is followed by the gather launch
   if (fuse_route_permute(L)) {
     const PermuteArgs p = permute_args(d, L, ids, sc, counts, offsets, rows, inv, W, true);
     const GatherArgs g = gather_args(d, L, x, rows, W + L.a_perm, W);
     const bool fg = fuse_route_gather(d, L);
     FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s, &p, fg ? &g : nullptr));
     if (!fg) FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
+    plan_two_back = !fg;
   } else {
     FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
     FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s,
                           /*with_plan=*/true));
   }
   FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s,
-                        /*plan_done=*/true, /*fused_out=*/out, ids, inv));
+                        /*plan_done=*/true, /*fused_out=*/out, ids, inv, plan_two_back));
   if (L.swap) return FMOE_OK;  // combined by combine_partials
   return combine_impl(d, y, inv, out, s);
 }

@@ -143,6 +143,8 @@ struct GemmArgs {
   int rows_per_expert;     // weight rows per expert in map_w (2I or H)
   int chunk_rows;
   int nstages;             // shared-memory pipeline depth (gemm_stages)
+  int prefetch_w;          // 1: the chunk list was written at least two launches earlier,
+                           // so weight tiles may be loaded before griddepcontrol.wait
   uint64_t wait_budget_ns;
 };
 // gemm = 1 (w13, gate/up) or 2 (w2); fp8 selects kind::f8f6f4 vs kind::f16.

@@ -137,13 +137,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // The first contraction's work list is written by the kernel right before it, so it
-  // waits here.  The second contraction's work list was written at least two kernels
-  // earlier, which has completed by the time this grid starts (every kernel triggers
-  // its dependents only after its own wait), so its weight tiles are prefetched before
+  // When the work list was written by the kernel right before this one it waits here.
+  // When it was written at least two kernels earlier (a.prefetch_w: always for the second
+  // contraction, and for the first one when the gather runs as its own launch), that
+  // kernel has completed by the time this grid starts (every kernel triggers its
+  // dependents only after its own wait), so the weight tiles are prefetched before
   // waiting for the activations.
-  constexpr bool kPrefetch = (kGemm == 2);
-  if constexpr (!kPrefetch) griddep_wait();
+  const bool prefetch = a.prefetch_w != 0;
+  if (!prefetch) griddep_wait();
   if (threadIdx.x == 0) {
     ctl.n_chunks = a.hdr->n_chunks;
     ctl.split = kSwap ? (kGemm == 1 ? a.hdr->split1 : a.hdr->split2) : 1;
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if constexpr (!kPrefetch) {
+  if (!prefetch) {
     if (threadIdx.x == 0) griddep_launch_dependents();
   }
 
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 
       Cursor cur;
       cursor_start(cur);
-      if constexpr (kPrefetch) {
+      if (prefetch) {
         // weights of the first stages (fresh stages: nothing to wait for)
         Cursor first = cur;
         int npre = 0;
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             mbar_wait(&ctl.full[s], (issued_parity >> s) & 1u, &dummy, a.status, budget);
           }
       }
-    } else if (kPrefetch) {
+    } else if (prefetch) {
       // lanes that do not produce still order their later reads after the wait
       griddep_wait();
     }
@@ -341,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    if constexpr (kPrefetch) griddep_wait();  // scales and routing weights of this call
+    if (prefetch) griddep_wait();  // scales and routing weights of this call
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
     int acc = 0;

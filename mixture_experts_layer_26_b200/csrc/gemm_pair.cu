@@ -250,15 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     tmem_alloc_pair(&ctl.tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
-  // As in the one-CTA kernel: the first contraction waits for its work list here; the
-  // second one's list was written at least two kernels earlier, so it prefetches weights.
-  constexpr bool kPrefetch = (kGemm == 2);
-  if constexpr (!kPrefetch) griddep_wait();
+  // As in the one-CTA kernel: weight tiles are prefetched before waiting on the previous
+  // kernel when the work list was written at least two kernels earlier (a.prefetch_w).
+  const bool prefetch = a.prefetch_w != 0;
+  if (!prefetch) griddep_wait();
   if (threadIdx.x == 0) ctl.n_chunks = a.hdr->n_chunks;
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers initialised, the pair's TMEM allocated
   tc_fence_after();
-  if constexpr (!kPrefetch) {
+  if (!prefetch) {
     if (threadIdx.x == 0) griddep_launch_dependents();
   }
 
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           if (u < total) t = decode_pair_unit(u, a.chunks, tiles);
         }
       };
-      if constexpr (kPrefetch) {
+      if (prefetch) {
         // weights of the first stages (fresh stages: nothing to wait for)
         const long u_first = u;
         const PairUnit t_first = t;
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
         }
       }
       ctl.issued = issued;
-    } else if (kPrefetch) {
+    } else if (prefetch) {
       griddep_wait();
     }
   } else if (warp == 1) {
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    if constexpr (kPrefetch) griddep_wait();  // scales and routing weights of this call
+    if (prefetch) griddep_wait();  // scales and routing weights of this call
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
     const int r = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the unit
     int acc = 0;
