@@ -5,6 +5,9 @@ consumes. It contains none of the layer's arithmetic (no routing, no permutation
 no contraction). It is shared by the GPU tests, the benchmark and the CPU-side
 tests, so that both sides of every parity check read identical bytes.
 
+Shared experts (n_shared > 0) are generated like routed ones and stored after them:
+w13 / w2 / scales have E + n_shared experts, router_w has E rows.
+
 Workloads (the MoE shapes named for the method "Mixture-of-Experts kernel
 engineering on Amazon SageMaker AI": Mixtral-like and DeepSeek-V3-like experts,
 a large expert dimension of 8192 for the Swap-AB case, and a prefill batch):
@@ -45,10 +48,16 @@ class MoEShape:
     name: str = ""
     # group-limited sigmoid routing: (n_group, topk_group, routed_scaling); None = softmax
     grouped: Optional[tuple] = None
+    # shared experts (every token, weight 1), stored after the E routed experts
+    n_shared: int = 0
 
     @property
     def R(self) -> int:
-        return self.T * self.top_k
+        return self.T * (self.top_k + self.n_shared)
+
+    @property
+    def E_all(self) -> int:
+        return self.E + self.n_shared
 
 
 # The five workloads.  Decode workloads list every batch size they are run at.
@@ -64,10 +73,12 @@ WORKLOADS = {
     # the same Mixtral-like shapes with bf16 weights and activations
     "mixtral_bf16_decode": dict(Ts=(1, 8, 32, 64), H=4096, I=14336, E=8, top_k=2, wdtype="bf16"),
     "prefill_bf16": dict(Ts=(4096,), H=4096, I=14336, E=8, top_k=2, wdtype="bf16"),
-    # DeepSeek-V3-like shapes with its group-limited sigmoid router: 8 groups of 32
-    # experts, 4 groups kept, routed scaling 2.5, a seeded selection bias
+    # DeepSeek-V3-like shapes with its group-limited sigmoid router (8 groups of 32
+    # experts, 4 groups kept, routed scaling 2.5, a seeded selection bias) and its one
+    # shared expert of the routed experts' shape
     "dsv3_grouped_fp8_decode": dict(Ts=(16, 64, 256), H=7168, I=2048, E=256, top_k=8,
-                                    wdtype="fp8", router_std=1.0, grouped=(8, 4, 2.5)),
+                                    wdtype="fp8", router_std=1.0, grouped=(8, 4, 2.5),
+                                    n_shared=1),
 }
 
 
@@ -127,11 +138,11 @@ def make_weights(s: MoEShape, seed: int = 0):
     """Expert weights in the layer's storage format, generated one expert at a time."""
     fp8 = s.wdtype == "fp8"
     dt = torch.uint8 if fp8 else torch.bfloat16
-    w13 = torch.empty(s.E, 2 * s.I, s.H, dtype=dt)
-    w2 = torch.empty(s.E, s.H, s.I, dtype=dt)
-    s13 = torch.ones(s.E, dtype=torch.float32)
-    s2 = torch.ones(s.E, dtype=torch.float32)
-    for e in range(s.E):
+    w13 = torch.empty(s.E_all, 2 * s.I, s.H, dtype=dt)
+    w2 = torch.empty(s.E_all, s.H, s.I, dtype=dt)
+    s13 = torch.ones(s.E_all, dtype=torch.float32)
+    s2 = torch.ones(s.E_all, dtype=torch.float32)
+    for e in range(s.E_all):
         a = torch.randn(2 * s.I, s.H, generator=_gen(seed, 3, e), dtype=torch.float32)
         a *= 1.0 / math.sqrt(s.H)
         b = torch.randn(s.H, s.I, generator=_gen(seed, 4, e), dtype=torch.float32)

@@ -56,6 +56,8 @@ Readings where the pages are silent (each is listed in the design doc):
 The grouped sigmoid routing of router_grouped (a later variant of step 1-3 for the
 DeepSeek-V3-like shapes; the pages name DeepSeek-V3 but do not describe its router) is
 taken from DeepSeek-V3's published design; its readings D1-D5 are listed there.
+Shared experts (DeepSeek-V3's always-active experts; readings S1-S2 at
+append_shared) are experts E..E+n_shared-1 that every token uses with weight 1.
 """
 from __future__ import annotations
 
@@ -226,6 +228,26 @@ def grouped_select(logits, top_k, n_group, topk_group, bias=None, routed_scaling
     return ids, w.astype(np.float32), s, sb
 
 
+def append_shared(ids: np.ndarray, w: np.ndarray, E: int, n_shared: int):
+    """Routing slots with the shared experts appended (DeepSeek-V3's published design
+    adds the output of its always-active shared expert to the routed mixture).
+
+    S1 shared expert s is expert E+s of w13/w2 (and of their scales); every token
+       uses it with weight exactly 1 (fp32), outside the renormalisation of the routed
+       weights and outside routed_scaling;
+    S2 it takes slot k+s of the token, after the k routed slots, so the combine adds
+       it last; its rows belong to the layer like any expert's (one per-tensor scale
+       for h over all rows).
+    Returns ids [T, k+n_shared] int32 and w [T, k+n_shared] float32."""
+    if n_shared == 0:
+        return ids, w
+    T = ids.shape[0]
+    sid = np.broadcast_to(np.arange(E, E + n_shared, dtype=np.int32), (T, n_shared))
+    sw = np.ones((T, n_shared), np.float32)
+    return (np.concatenate([ids, sid], axis=1).astype(np.int32),
+            np.concatenate([w, sw], axis=1).astype(np.float32))
+
+
 # --------------------------------------------------------------------------------------
 # Step 4: permutation ("data shuffling": [readmex] opening; irregular access and
 # dynamic per-expert batch sizes: [n1n] "The Core Bottlenecks of MoE Inference").
@@ -358,11 +380,13 @@ def combine(y, inv_perm, T, top_k):
 
 
 def fused_moe(x_bits, wr_bits, w13, w2, top_k, fp8=True, w13_scale=None, w2_scale=None,
-              a1_scale=0.0, a2_scale=0.0, grouped=None):
+              a1_scale=0.0, a2_scale=0.0, grouped=None, n_shared=0):
     """The whole layer on host arrays.  x_bits [T,H] / wr_bits [E,H] are bf16 bit
-    patterns (uint16); w13 [E,2I,H], w2 [E,H,I] are e4m3 codes (uint8) or bf16 bits.
-    grouped: None for softmax top-k routing, else the router_grouped parameters.
-    Returns a dict with every intermediate the GPU path also exposes."""
+    patterns (uint16); w13 [E+n_shared,2I,H], w2 [E+n_shared,H,I] are e4m3 codes
+    (uint8) or bf16 bits.  grouped: None for softmax top-k routing, else the
+    router_grouped parameters.  n_shared: shared experts after the E routed ones.
+    Returns a dict with every intermediate the GPU path also exposes; topk_ids /
+    topk_w include the shared slots."""
     x_bits = np.asarray(x_bits)
     T, H = x_bits.shape
     E = wr_bits.shape[0]
@@ -371,11 +395,13 @@ def fused_moe(x_bits, wr_bits, w13, w2, top_k, fp8=True, w13_scale=None, w2_scal
         ids, w, logits = router(x_bits, wr_bits, top_k)
     else:   # dict(n_group=, topk_group=, bias=, routed_scaling=)
         ids, w, logits, _ = router_grouped(x_bits, wr_bits, top_k, **grouped)
-    counts, offsets, sorted_rows, inv_perm = permute(ids, E)
-    a_perm, s1, inv1, amax_x = permute_quant(x_bits, sorted_rows, top_k, fp8, a1_scale)
-    y, h, hq, s2 = experts(a_perm, offsets, sorted_rows, w, w13, w2, H, I, E, fp8, s1,
+    ids, w = append_shared(ids, w, E, n_shared)
+    k_all, E_all = top_k + n_shared, E + n_shared
+    counts, offsets, sorted_rows, inv_perm = permute(ids, E_all)
+    a_perm, s1, inv1, amax_x = permute_quant(x_bits, sorted_rows, k_all, fp8, a1_scale)
+    y, h, hq, s2 = experts(a_perm, offsets, sorted_rows, w, w13, w2, H, I, E_all, fp8, s1,
                            w13_scale, w2_scale, a2_scale)
-    out, out64 = combine(y, inv_perm, T, top_k)
+    out, out64 = combine(y, inv_perm, T, k_all)
     return dict(topk_ids=ids, topk_w=w, logits=logits, amax_x=amax_x, counts=counts,
                 offsets=offsets, sorted_rows=sorted_rows, inv_perm=inv_perm,
                 a_perm=a_perm, s1=s1, inv1=inv1, h=h, hq=hq, s2=s2, y=y,

@@ -51,8 +51,12 @@ def exact_logits(x_bits, wr_bits):
     return [[math.fsum(a * b for a, b in zip(xt, we)) for we in w] for xt in x]
 
 
-def brute_force(x_bits, wr_bits, w13, w2, top_k, fp8, w13_scale=None, w2_scale=None):
-    """Returns dict(ids, weights, out [T][H] floats (bf16 values), h [(t,j)] lists)."""
+def brute_force(x_bits, wr_bits, w13, w2, top_k, fp8, w13_scale=None, w2_scale=None,
+                n_shared=0):
+    """Returns dict(ids, weights, out [T][H] floats (bf16 values), h [(t,j)] lists).
+
+    n_shared: experts E..E+n_shared-1 of w13/w2 join every token after its k routed
+    experts with weight 1 (DeepSeek-V3's always-active shared experts)."""
     x = _bf16_bits_to_float(x_bits).tolist()
     T, H = len(x), len(x[0])
     E = len(wr_bits)
@@ -65,8 +69,8 @@ def brute_force(x_bits, wr_bits, w13, w2, top_k, fp8, w13_scale=None, w2_scale=N
         z = math.fsum(p)
         p = [v / z for v in p]                       # softmax over all experts
         zs = math.fsum(p[e] for e in order)
-        ids.append(order)
-        weights.append([_f32(p[e] / zs) for e in order])   # stored as fp32
+        ids.append(order + [E + i for i in range(n_shared)])
+        weights.append([_f32(p[e] / zs) for e in order] + [1.0] * n_shared)   # fp32
 
     if fp8:
         W13 = _e4m3_to_float(w13).tolist()

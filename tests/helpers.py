@@ -39,7 +39,7 @@ def run_oracle(oracle_mod, inp, a1_scale=0.0, a2_scale=0.0):
     return oracle_mod.fused_moe(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], d["top_k"],
                                 fp8=d["fp8"], w13_scale=d["w13_scale"],
                                 w2_scale=d["w2_scale"], a1_scale=a1_scale, a2_scale=a2_scale,
-                                grouped=grouped_args(inp))
+                                grouped=grouped_args(inp), n_shared=inp.shape.n_shared)
 
 
 def bf16_bits_to_float(bits) -> np.ndarray:

@@ -462,3 +462,63 @@ def test_grouped_routing_matches_bruteforce(seed, T, E, G, M, k):
         gscore = np.sort(groups, axis=1)[:, -1] + np.sort(groups, axis=1)[:, -2]
         kept = set(sorted(range(G), key=lambda g: (-gscore[g], g))[:M])
         assert {int(e) // eg for e in ids[t]} <= kept
+
+
+# ----------------------------------------------------------------------------- shared experts
+
+@pytest.mark.parametrize("seed,T,H,I,E,k,ns,wdtype", [
+    (6, 3, 256, 256, 4, 2, 1, "fp8"),
+    (7, 2, 256, 128, 4, 1, 2, "bf16"),
+    (8, 3, 256, 256, 1, 1, 1, "fp8"),   # one routed expert (weight 1) plus one shared
+])
+def test_shared_experts_match_bruteforce(seed, T, H, I, E, k, ns, wdtype):
+    s = tiny_shape(T, H, I, E, k, wdtype, n_shared=ns)
+    inp = minp.make_inputs(s, seed=seed)
+    d = np_inputs(inp)
+    r = run_oracle(O, inp)
+    b = brute_force(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], k, d["fp8"],
+                    d["w13_scale"], d["w2_scale"], n_shared=ns)
+    assert r["topk_ids"].tolist() == b["ids"]
+    assert np.allclose(r["topk_w"], np.array(b["weights"]), rtol=1e-6, atol=0)
+    assert np.array_equal(r["counts"][E:], np.full(ns, T))          # every token, once each
+    hb = np.array([b["h"][(t, j)] for t in range(T) for j in range(k + ns)], np.float32)
+    h_or = r["h"][r["inv_perm"]]
+    assert np.abs(h_or - hb).max() <= 1e-6 * np.abs(hb).max()
+    out_o = bf16_bits_to_float(r["out"])
+    assert max_rel_err(out_o, np.array(b["out"])) <= 2.0 ** -8
+
+
+def test_shared_slots_follow_the_routed_ones_with_weight_one():
+    # grouped routing with routed_scaling 2.5: routed weights sum to 2.5, the shared
+    # slots keep weight exactly 1 and come last, in expert order
+    s = tiny_shape(6, 256, 128, 16, 3, "fp8", router_std=1.0, grouped=(4, 2, 2.5), n_shared=2)
+    inp = minp.make_inputs(s, seed=3)
+    r = run_oracle(O, inp)
+    ids, w = r["topk_ids"], r["topk_w"]
+    assert ids.shape == (6, 5) and w.shape == (6, 5)
+    assert np.all(ids[:, 3:] == np.array([16, 17])) and np.all(ids[:, :3] < 16)
+    assert np.all(w[:, 3:] == np.float32(1.0))
+    assert np.allclose(w[:, :3].sum(axis=1), 2.5, rtol=1e-6)
+    assert np.all(r["counts"][16:] == 6)
+
+
+def test_shared_expert_adds_a_dense_gated_mlp():
+    """bf16 format (no per-tensor scale couples the rows): the layer's unrounded output
+    with the shared expert minus the output without it is the shared expert's dense
+    gated MLP of every token, computed here with torch in float64."""
+    T, H, I, E, k = 5, 256, 128, 6, 2
+    s1 = tiny_shape(T, H, I, E, k, "bf16", n_shared=1)
+    inp = minp.make_inputs(s1, seed=9)
+    d = np_inputs(inp)
+    with_s = run_oracle(O, inp)
+    without = O.fused_moe(d["x_bits"], d["wr_bits"], d["w13"][:E], d["w2"][:E], k, fp8=False)
+    assert np.array_equal(with_s["topk_ids"][:, :k], without["topk_ids"])
+    diff = with_s["out64"] - without["out64"]
+    x = torch.from_numpy(bf16_bits_to_float(d["x_bits"]).astype(np.float64))
+    w13 = torch.from_numpy(bf16_bits_to_float(d["w13"][E]).astype(np.float64))
+    w2 = torch.from_numpy(bf16_bits_to_float(d["w2"][E]).astype(np.float64))
+    gu = x @ w13.T
+    h = (torch.nn.functional.silu(gu[:, :I]) * gu[:, I:]).to(torch.float32)
+    h = h.to(torch.bfloat16).to(torch.float64)                      # R7: h rounded to bf16
+    y = (h @ w2.T).numpy()
+    assert np.abs(diff - y).max() <= 1e-9 * np.abs(y).max()
