@@ -164,6 +164,26 @@ def np_inputs(inp: minp.MoEInputs):
                 w2_scale=None if inp.w2_scale is None else inp.w2_scale.numpy(), fp8=fp8)
 
 
+def oracle_grouped(inp: minp.MoEInputs):
+    """The oracle's grouped-routing arguments for these inputs (None: softmax)."""
+    s = inp.shape
+    if s.grouped is None:
+        return None
+    return dict(n_group=s.grouped[0], topk_group=s.grouped[1], routed_scaling=s.grouped[2],
+                bias=inp.router_bias.numpy())
+
+
+def routing_desc(inp: minp.MoEInputs, device):
+    """The C-ABI routing descriptor of these inputs (None: softmax, no shared experts)."""
+    from mixture_experts_layer_26_b200 import capi
+    s = inp.shape
+    if s.grouped is not None:
+        return capi.make_routing(*s.grouped, inp.router_bias.to(device), n_shared=s.n_shared)
+    if s.n_shared:
+        return capi.make_softmax_routing(s.n_shared)
+    return None
+
+
 def reduce_max(dist, v: float, device) -> float:
     """Max of a per-rank scalar over all ranks (identity without a process group)."""
     if dist is None:
@@ -186,7 +206,8 @@ def oracle_full_pass(inp):
     d = np_inputs(inp)
     t0 = time.perf_counter()
     r = O.fused_moe(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], inp.shape.top_k, fp8=d["fp8"],
-                    w13_scale=d["w13_scale"], w2_scale=d["w2_scale"])
+                    w13_scale=d["w13_scale"], w2_scale=d["w2_scale"], grouped=oracle_grouped(inp),
+                    n_shared=inp.shape.n_shared)
     return time.perf_counter() - t0, int((r["counts"] > 0).sum())
 
 
@@ -200,12 +221,18 @@ class OracleSlices:
         s = inp.shape
         t0 = time.perf_counter()
         d = self.d
-        ids, w, _ = O.router(d["x_bits"], d["wr_bits"], s.top_k)
-        counts, offsets, rows, inv = O.permute(ids, s.E)
-        a_perm, s1, _, _ = O.permute_quant(d["x_bits"], rows, s.top_k, d["fp8"])
+        grouped = oracle_grouped(inp)
+        if grouped is None:
+            ids, w, _ = O.router(d["x_bits"], d["wr_bits"], s.top_k)
+        else:
+            ids, w, _, _ = O.router_grouped(d["x_bits"], d["wr_bits"], s.top_k, **grouped)
+        ids, w = O.append_shared(ids, w, s.E, s.n_shared)
+        K = s.top_k + s.n_shared
+        counts, offsets, rows, inv = O.permute(ids, s.E_all)
+        a_perm, s1, _, _ = O.permute_quant(d["x_bits"], rows, K, d["fp8"])
         self.prep = (ids, w, counts, offsets, rows, inv, a_perm, s1)
         self.fixed_s = time.perf_counter() - t0
-        self.touched = [e for e in range(s.E) if counts[e] > 0]
+        self.touched = [e for e in range(s.E_all) if counts[e] > 0]
         self.i = 0
 
     def step(self):
@@ -216,14 +243,14 @@ class OracleSlices:
         offs = np.zeros_like(offsets)
         offs[e + 1:] = offsets[e + 1] - offsets[e]
         r0, r1 = offsets[e], offsets[e + 1]
-        O.experts(a_perm[r0:r1], offs, rows[r0:r1], w, d["w13"], d["w2"], s.H, s.I, s.E, d["fp8"],
-                  s1, d["w13_scale"], d["w2_scale"])
+        O.experts(a_perm[r0:r1], offs, rows[r0:r1], w, d["w13"], d["w2"], s.H, s.I, s.E_all,
+                  d["fp8"], s1, d["w13_scale"], d["w2_scale"])
 
     def combine_seconds(self):
         s = self.inp.shape
         y = np.zeros((s.R, s.H))
         t0 = time.perf_counter()
-        self.O.combine(y, self.prep[5], s.T, s.top_k)
+        self.O.combine(y, self.prep[5], s.T, s.top_k + s.n_shared)
         return time.perf_counter() - t0
 
 
@@ -266,10 +293,15 @@ def run_reference(args, rank):
 # --------------------------------------------------------------------------- GPU arm
 
 def workload_config(s, variant):
-    weights = 3 * s.H * s.I * s.E * (1 if s.wdtype == "fp8" else 2)
-    return {"workload": f"{s.name}: H={s.H} I={s.I} E={s.E} top_k={s.top_k} T={s.T} "
+    weights = 3 * s.H * s.I * s.E_all * (1 if s.wdtype == "fp8" else 2)
+    routing = "softmax top-k" if s.grouped is None else \
+        (f"grouped sigmoid: {s.grouped[0]} groups, {s.grouped[1]} kept, "
+         f"routed scaling {s.grouped[2]}, selection bias")
+    shared = f" + {s.n_shared} shared" if s.n_shared else ""
+    return {"workload": f"{s.name}: H={s.H} I={s.I} E={s.E}{shared} top_k={s.top_k} T={s.T} "
                         f"({s.wdtype} weights)",
-            "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.top_k, "variant": variant,
+            "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.top_k, "n_shared": s.n_shared,
+            "routing": routing, "variant": variant,
             "l2": f"inputs larger than L2: expert weights {weights / 1e9:.2f} GB vs "
                   f"{L2_BYTES / 2 ** 20:.0f} MB L2, no flush",
             "parallelism": "replicas (one independent layer per GPU)"}
@@ -292,7 +324,8 @@ def run_ours(args, rank, world, local_rank):
     w13, w2 = inp.w13.to(dev), inp.w2.to(dev)
     s13 = inp.w13_scale.to(dev) if fp8 else None
     s2 = inp.w2_scale.to(dev) if fp8 else None
-    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, args.variant)
+    routing = routing_desc(inp, dev)
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, args.variant, routing=routing)
     ws = capi.alloc_workspace(dims, dev)
     sc = capi.make_scales(s13, s2)
     out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device=dev)
@@ -358,8 +391,8 @@ def run_ours(args, rank, world, local_rank):
     R = s.R
     ids_d = torch.empty(R, dtype=torch.int32, device=dev)
     tw_d = torch.empty(R, dtype=torch.float32, device=dev)
-    counts_d = torch.empty(s.E, dtype=torch.int32, device=dev)
-    offs_d = torch.empty(s.E + 1, dtype=torch.int32, device=dev)
+    counts_d = torch.empty(s.E_all, dtype=torch.int32, device=dev)
+    offs_d = torch.empty(s.E_all + 1, dtype=torch.int32, device=dev)
     rows_d = torch.empty(R, dtype=torch.int32, device=dev)
     inv_d = torch.empty(R, dtype=torch.int32, device=dev)
     aperm_d = torch.empty(R, s.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)

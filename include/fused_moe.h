@@ -36,8 +36,8 @@
  *  - Argument checks run before any CUDA call and return synchronously:
  *      FMOE_ERR_INVALID_ARG  null dims / pointer, T < 0, H, I < 1, E < 1 or > 256,
  *                            top_k < 1 or > E, unknown wdtype / variant / routing
- *                            mode, routing parameters outside their ranges, FP8
- *                            without weight scales
+ *                            mode, routing parameters outside their ranges (n_shared
+ *                            outside 0..8 included), FP8 without weight scales
  *      FMOE_ERR_UNSUPPORTED  H % 256 != 0, I % 128 != 0, H > 16384, a device pointer
  *                            not 16-byte aligned, sizes whose element counts exceed
  *                            2^31
@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define FUSED_MOE_ABI_VERSION 2
+#define FUSED_MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define FMOE_API __attribute__((visibility("default")))
@@ -114,12 +114,22 @@ typedef enum {
  *    weights = s / (sum of the chosen s) * routed_scaling. */
 typedef enum { FMOE_ROUTE_SOFTMAX = 0, FMOE_ROUTE_SIGMOID_GROUPED = 1 } fmoe_route_mode;
 
+/* Shared experts (either mode; DeepSeek-V3's always-active experts): n_shared = S > 0
+ * appends experts E..E+S-1, which every token uses with weight exactly 1 (outside the
+ * renormalisation and outside routed_scaling).  They take slots k..k+S-1 of each token,
+ * after its k routed slots, so with K = k + S:
+ *   w13 [E+S, 2I, H], w2 [E+S, H, I] and the FP8 weight scales [E+S] hold the routed
+ *   experts first and the shared ones after them; router_w and bias stay [E];
+ *   topk_ids / topk_w are [T, K]; counts [E+S]; offsets [E+S+1]; sorted_rows,
+ *   inv_perm [T*K]; a_perm, y_perm [T*K, H]; the combine sums the K slots in order.
+ * Shared rows take part in the per-tensor scale of h like every other row. */
 typedef struct {
   int32_t mode;           /* fmoe_route_mode */
   int32_t n_group;        /* SIGMOID_GROUPED: 1..32 groups, E % n_group == 0, E/n_group >= 2 */
   int32_t topk_group;     /* SIGMOID_GROUPED: 1..n_group, topk_group * E/n_group >= top_k */
   float routed_scaling;   /* SIGMOID_GROUPED: > 0, multiplies the renormalised weights */
   const float* bias;      /* SIGMOID_GROUPED: [E] device fp32 selection bias, or NULL */
+  int32_t n_shared;       /* 0..8 shared experts (any mode) */
 } fmoe_routing;
 
 typedef struct {
@@ -130,7 +140,8 @@ typedef struct {
   int32_t top_k;    /* experts per token */
   int32_t wdtype;   /* fmoe_wdtype */
   int32_t variant;  /* fmoe_variant */
-  const fmoe_routing* routing; /* host pointer, read during the call; NULL = softmax */
+  const fmoe_routing* routing; /* host pointer, read during the call; NULL = softmax,
+                                  no shared experts */
 } fmoe_dims;
 
 typedef struct {

@@ -46,7 +46,7 @@ FMOE_ROUTE_SOFTMAX, FMOE_ROUTE_SIGMOID_GROUPED = 0, 1
 
 class FmoeRouting(ctypes.Structure):
     _fields_ = [("mode", c_int32), ("n_group", c_int32), ("topk_group", c_int32),
-                ("routed_scaling", c_float), ("bias", c_void_p)]
+                ("routed_scaling", c_float), ("bias", c_void_p), ("n_shared", c_int32)]
 
 
 class FmoeDims(ctypes.Structure):
@@ -128,12 +128,18 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_routing(n_group: int, topk_group: int, routed_scaling: float = 1.0,
-                 bias: Optional[torch.Tensor] = None) -> FmoeRouting:
-    """Group-limited sigmoid routing (DeepSeek-V3 style); bias: [E] fp32 device tensor."""
+                 bias: Optional[torch.Tensor] = None, n_shared: int = 0) -> FmoeRouting:
+    """Group-limited sigmoid routing (DeepSeek-V3 style); bias: [E] fp32 device tensor;
+    n_shared shared experts stored after the E routed ones."""
     r = FmoeRouting(FMOE_ROUTE_SIGMOID_GROUPED, n_group, topk_group, float(routed_scaling),
-                    _ptr(bias))
+                    _ptr(bias), int(n_shared))
     r._bias_ref = bias  # keep the tensor alive with the descriptor
     return r
+
+
+def make_softmax_routing(n_shared: int = 0) -> FmoeRouting:
+    """Softmax top-k routing with n_shared shared experts after the E routed ones."""
+    return FmoeRouting(FMOE_ROUTE_SOFTMAX, 0, 0, 1.0, None, int(n_shared))
 
 
 def make_dims(T: int, H: int, I: int, E: int, top_k: int, fp8: bool, variant: str = "auto",
@@ -267,27 +273,35 @@ def fused_moe_profile(dims, x, router_w, w13, w2, scales, out, ws, stream=None):
 class FusedMoE:
     """The whole layer on device tensors, with its own workspace.
 
-    x [T,H] bf16, router_w [E,H] bf16, w13 [E,2I,H] and w2 [E,H,I] as uint8 e4m3
-    bytes (with w13_scale, w2_scale [E] fp32) or bf16.  Returns out [T,H] bf16."""
+    x [T,H] bf16, router_w [E,H] bf16, w13 [E+S,2I,H] and w2 [E+S,H,I] as uint8 e4m3
+    bytes (with w13_scale, w2_scale [E+S] fp32) or bf16, where S = w13.shape[0] - E
+    shared experts follow the E routed ones.  routing: a descriptor from make_routing
+    or make_softmax_routing (default: softmax with the S shared experts).
+    Returns out [T,H] bf16."""
 
     def __init__(self, router_w, w13, w2, top_k, w13_scale=None, w2_scale=None,
-                 a1_scale=0.0, a2_scale=0.0, variant="auto"):
+                 a1_scale=0.0, a2_scale=0.0, variant="auto", routing=None):
         self.router_w, self.w13, self.w2 = router_w, w13, w2
         self.top_k, self.variant = top_k, variant
         self.w13_scale, self.w2_scale = w13_scale, w2_scale
         self.scales = make_scales(w13_scale, w2_scale, a1_scale, a2_scale)
+        n_shared = w13.shape[0] - router_w.shape[0]
+        if routing is None and n_shared > 0:
+            routing = make_softmax_routing(n_shared)
+        if n_shared != (routing.n_shared if routing is not None else 0):
+            raise ValueError("w13 holds E + n_shared experts: n_shared must match the routing")
+        self.routing = routing
         self._ws = {}
 
     def workspace(self, T: int) -> torch.Tensor:
         if T not in self._ws:
-            dims = make_dims(T, self.w13.shape[2], self.w13.shape[1] // 2, self.w13.shape[0],
-                             self.top_k, self.w13.dtype == torch.uint8, self.variant)
-            self._ws[T] = alloc_workspace(dims, self.w13.device)
+            self._ws[T] = alloc_workspace(self.dims(T), self.w13.device)
         return self._ws[T]
 
     def dims(self, T: int) -> FmoeDims:
-        return make_dims(T, self.w13.shape[2], self.w13.shape[1] // 2, self.w13.shape[0],
-                         self.top_k, self.w13.dtype == torch.uint8, self.variant)
+        return make_dims(T, self.w13.shape[2], self.w13.shape[1] // 2, self.router_w.shape[0],
+                         self.top_k, self.w13.dtype == torch.uint8, self.variant,
+                         routing=self.routing)
 
     def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
         T = x.shape[0]

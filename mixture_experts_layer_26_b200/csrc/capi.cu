@@ -35,6 +35,12 @@ struct Layout {
   size_t total = 0;
 };
 
+// Shared experts: S = n_shared; every token has K = top_k + S slots and the expert
+// tensors hold E + S experts.
+inline int shared_of(const fmoe_dims& d) { return d.routing != nullptr ? d.routing->n_shared : 0; }
+inline int slots_of(const fmoe_dims& d) { return d.top_k + shared_of(d); }
+inline int experts_all(const fmoe_dims& d) { return d.E + shared_of(d); }
+
 fmoe_status check_dims(const fmoe_dims* d) {
   if (d == nullptr) return FMOE_ERR_INVALID_ARG;
   if (d->T < 0 || d->H < 1 || d->I < 1 || d->E < 1 || d->E > kMaxExperts || d->top_k < 1 ||
@@ -47,6 +53,7 @@ fmoe_status check_dims(const fmoe_dims* d) {
     const fmoe_routing& r = *d->routing;
     if (r.mode != FMOE_ROUTE_SOFTMAX && r.mode != FMOE_ROUTE_SIGMOID_GROUPED)
       return FMOE_ERR_INVALID_ARG;
+    if (r.n_shared < 0 || r.n_shared > kMaxShared) return FMOE_ERR_INVALID_ARG;
     if (r.mode == FMOE_ROUTE_SIGMOID_GROUPED) {
       if (r.n_group < 1 || r.n_group > 32 || d->E % r.n_group != 0 || d->E / r.n_group < 2)
         return FMOE_ERR_INVALID_ARG;
@@ -59,19 +66,19 @@ fmoe_status check_dims(const fmoe_dims* d) {
     }
   }
   if (d->H % 256 != 0 || d->I % 128 != 0 || d->H > 16384) return FMOE_ERR_UNSUPPORTED;
-  const int64_t R = static_cast<int64_t>(d->T) * d->top_k;
+  const int64_t R = static_cast<int64_t>(d->T) * slots_of(*d);
   const int64_t lim = int64_t(1) << 31;
   if (R * std::max<int64_t>(d->H, 2 * int64_t(d->I)) >= lim) return FMOE_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(d->E) * 2 * d->I >= lim || static_cast<int64_t>(d->E) * d->H >= lim)
-    return FMOE_ERR_UNSUPPORTED;
+  const int64_t ea = experts_all(*d);
+  if (ea * 2 * d->I >= lim || ea * d->H >= lim) return FMOE_ERR_UNSUPPORTED;
   return FMOE_OK;
 }
 
 Layout make_layout(const fmoe_dims& d) {
   Layout L;
   L.fp8 = d.wdtype == FMOE_FP8_E4M3;
-  const int T = d.T, H = d.H, I = d.I, E = d.E;
-  const int R = T * d.top_k;
+  const int T = d.T, H = d.H, I = d.I, E = experts_all(d);
+  const int R = T * slots_of(d);
   L.R = R;
   int variant = d.variant;
   if (variant == FMOE_VARIANT_AUTO) {
@@ -288,6 +295,7 @@ fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const
   a.H = d.H;
   a.E = d.E;
   a.k = d.top_k;
+  a.n_shared = shared_of(d);
   a.num_sms = num_sms();
   a.mode = FMOE_ROUTE_SOFTMAX;
   a.routed_scaling = 1.f;
@@ -325,8 +333,8 @@ PermuteArgs permute_args(const fmoe_dims& d, const Layout& L, const int32_t* ids
   p.amax_part = reinterpret_cast<const float*>(W + L.amax_x);
   p.hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   p.R = L.R;
-  p.E = d.E;
-  p.k = d.top_k;
+  p.E = experts_all(d);
+  p.k = slots_of(d);
   p.fp8 = L.fp8 ? 1 : 0;
   p.a1_static = sc != nullptr ? sc->a1_scale : 0.f;
   p.with_plan = with_plan ? 1 : 0;
@@ -345,7 +353,7 @@ GatherArgs gather_args(const fmoe_dims& d, const Layout& L, const void* x, const
   g.status = &hdr->status;
   g.R = L.R;
   g.H = d.H;
-  g.k = d.top_k;
+  g.k = slots_of(d);
   g.fp8 = L.fp8 ? 1 : 0;
   return g;
 }
@@ -371,7 +379,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
                          const int32_t* inv = nullptr, bool plan_two_back = false) {
   const int sms = num_sms();
   const bool fp8 = L.fp8, swap = L.swap;
-  const int H = d.H, I = d.I, E = d.E, R = L.R;
+  const int H = d.H, I = d.I, E = experts_all(d), R = L.R;
   const int bk = fp8 ? 128 : 64;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   Chunk* chunks = reinterpret_cast<Chunk*>(W + L.chunks);
@@ -480,7 +488,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
     c.out = static_cast<uint16_t*>(fused_out);
     c.T = d.T;
     c.H = H;
-    c.k = d.top_k;
+    c.k = slots_of(d);
     c.E = E;
     c.fp8 = fp8 ? 1 : 0;
     FMOE_LAUNCH("combine_partials", launch_combine_partials(c, sms, s), s);
@@ -511,7 +519,7 @@ fmoe_status combine_impl(const fmoe_dims& d, const float* y, const int32_t* inv,
   c.out = static_cast<uint16_t*>(out);
   c.T = d.T;
   c.H = d.H;
-  c.k = d.top_k;
+  c.k = slots_of(d);
   FMOE_LAUNCH("combine", launch_combine(c, num_sms(), s), s);
   return FMOE_OK;
 }

@@ -48,7 +48,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 __global__ void __launch_bounds__(kEwThreads) finalize1_kernel(Finalize1Args a) {
-  __shared__ int offs[kMaxExperts + 1];
+  __shared__ int offs[kMaxAllExperts + 1];
   __shared__ float red[kEwThreads / 32];
   griddep_wait();
   griddep_launch_dependents();
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
 }
 
 __global__ void __launch_bounds__(kEwThreads) finalize2_kernel(Finalize2Args a) {
-  __shared__ int offs[kMaxExperts + 1];
+  __shared__ int offs[kMaxAllExperts + 1];
   griddep_wait();
   griddep_launch_dependents();
   for (int i = threadIdx.x; i <= a.E; i += kEwThreads) offs[i] = a.offsets[i];

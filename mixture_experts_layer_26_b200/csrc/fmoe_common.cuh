@@ -16,7 +16,10 @@ namespace fmoe {
 // Device status codes (same numbers as fmoe_status in include/fused_moe.h).
 enum : int32_t { ST_OK = 0, ST_TIMEOUT = 5, ST_BOUNDS = 6 };
 
-constexpr int kMaxExperts = 256;
+constexpr int kMaxExperts = 256;                          // routed experts
+constexpr int kMaxShared = 8;                             // shared experts
+constexpr int kMaxAllExperts = kMaxExperts + kMaxShared;  // rows of the expert tensors
+constexpr int kExpertsPerLane = (kMaxAllExperts + 31) / 32;  // one warp covers them all
 constexpr int kE4M3Max = 448;
 constexpr int kAmaxSlots = 4096;  // capacity of the per-CTA max |h| partials
 

@@ -95,7 +95,8 @@ struct RouterArgs {
   float* logits_g;         // [T, E] logits when the experts are split over CTAs
   int32_t* tile_counters;  // [kRouterMaxTiles] zero between calls (self-resetting)
   WsHeader* hdr;
-  int T, H, E, k;
+  int T, H, E, k;          // E routed experts, k routed slots per token
+  int n_shared;            // shared experts E..E+n_shared-1: slots k.., weight 1
   int num_sms;
   int experts_per_cta;     // set by the launcher
   // routing mode (fmoe_route_mode) and the grouped-sigmoid parameters

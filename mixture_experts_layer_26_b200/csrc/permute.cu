@@ -30,9 +30,9 @@ constexpr int kGatherThreads = 256;
 
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
   constexpr int kWarps = kPermThreads / 32;
-  __shared__ int cnt[kMaxExperts];
-  __shared__ int base[kMaxExperts + 1];
-  __shared__ int wc[kWarps * kMaxExperts];
+  __shared__ int cnt[kMaxAllExperts];
+  __shared__ int base[kMaxAllExperts + 1];
+  __shared__ int wc[kWarps * kMaxAllExperts];
   griddep_wait();
   griddep_launch_dependents();
   permute_body<kWarps>(a, wc, cnt, base);

@@ -33,10 +33,10 @@ __device__ int choose_split(int units, int kblocks, int smax, int sms) {
 __device__ void build_plan(const int* offsets, int E, int R, const PlanParams& p, WsHeader* hdr) {
   const int lane = threadIdx.x & 31;
   const int CH = p.chunk_rows;
-  int n[8], nch[8], s = 0;
+  int n[kExpertsPerLane], nch[kExpertsPerLane], s = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane * 8 + j;
+  for (int j = 0; j < kExpertsPerLane; ++j) {
+    const int e = lane * kExpertsPerLane + j;
     n[j] = 0;
     if (e < E) {
       const int lo = offsets[e], hi = offsets[e + 1];
@@ -55,8 +55,8 @@ __device__ void build_plan(const int* offsets, int E, int R, const PlanParams& p
   const int total = __shfl_sync(0xffffffffu, incl, 31);
   int cb = incl - s;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane * 8 + j;
+  for (int j = 0; j < kExpertsPerLane; ++j) {
+    const int e = lane * kExpertsPerLane + j;
     for (int c = 0; c < nch[j]; ++c) {
       const int idx = cb + c;
       if (idx >= p.max_chunks) {
@@ -159,12 +159,12 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
   }
   __syncthreads();
 
-  // exclusive scan of the counts: lane l owns experts 8l .. 8l+7
+  // exclusive scan of the counts: lane l owns experts l*kExpertsPerLane ..
   if (warp == 0) {
-    int v[8], s = 0;
+    int v[kExpertsPerLane], s = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
+    for (int j = 0; j < kExpertsPerLane; ++j) {
+      const int e = lane * kExpertsPerLane + j;
       v[j] = e < E ? cnt[e] : 0;
       s += v[j];
     }
@@ -176,8 +176,8 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
     }
     int run = incl - s;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane * 8 + j;
+    for (int j = 0; j < kExpertsPerLane; ++j) {
+      const int e = lane * kExpertsPerLane + j;
       if (e < E) {
         a.counts[e] = v[j];
         a.offsets[e] = run;

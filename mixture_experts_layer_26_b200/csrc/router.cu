@@ -17,7 +17,8 @@
 // One CTA (8 warps) handles TB tokens.  Their x rows are staged in shared memory with
 // 16-byte loads; each warp takes groups of EG experts and streams the router rows from
 // L2, so each x chunk read from shared memory feeds 8*EG FMAs.  Top-k is then one warp
-// per token: k rounds of a shuffle argmax over (logit desc, expert index asc).
+// per token: k rounds of a shuffle argmax over (logit desc, expert index asc); shared
+// experts, when present, fill the token's last slots with weight 1.
 #include <float.h>
 
 #include "permute_body.cuh"
@@ -252,8 +253,9 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
       }
     }
     float top0 = 0.f, wsum = 0.f;
-    float* wout = a.topk_w + static_cast<size_t>(tok) * a.k;
-    int32_t* iout = a.topk_ids + static_cast<size_t>(tok) * a.k;
+    const int K = a.k + a.n_shared;  // slots per token: k routed, then the shared experts
+    float* wout = a.topk_w + static_cast<size_t>(tok) * K;
+    int32_t* iout = a.topk_ids + static_cast<size_t>(tok) * K;
     for (int r = 0; r < a.k; ++r) {
       float bv = -INFINITY;
       int be = 0x7fffffff;
@@ -284,6 +286,11 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
     if (lane == 0) {
       const float scale = grouped ? a.routed_scaling : 1.f;
       for (int r = 0; r < a.k; ++r) wout[r] = grouped ? wout[r] / wsum * scale : wout[r] / wsum;
+      // shared experts: every token, weight exactly 1, after the routed slots
+      for (int r = 0; r < a.n_shared; ++r) {
+        iout[a.k + r] = a.E + r;
+        wout[a.k + r] = 1.f;
+      }
     }
   }
 
@@ -302,9 +309,11 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
     }
     __syncthreads();
     if (!is_final) return;
-    int* ps = reinterpret_cast<int*>(smem);  // reuse: wc[8*E], cnt[E], base[E+1]
-    permute_body<kRouterThreads / 32>(a.perm, ps, ps + (kRouterThreads / 32) * E,
-                                      ps + (kRouterThreads / 32 + 1) * E);
+    // reuse: wc[8*Ea], cnt[Ea], base[Ea+1] over all Ea experts (shared ones included)
+    const int Ea = a.perm.E;
+    int* ps = reinterpret_cast<int*>(smem);
+    permute_body<kRouterThreads / 32>(a.perm, ps, ps + (kRouterThreads / 32) * Ea,
+                                      ps + (kRouterThreads / 32 + 1) * Ea);
     if (a.fuse_gather) {
       __syncthreads();
       gather_rows(a.gather, warp, kRouterThreads / 32);
@@ -315,8 +324,8 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
 template <int TB, int EG>
 cudaError_t launch_tb(RouterArgs a, cudaStream_t s) {
   size_t smem = static_cast<size_t>(TB) * a.H * 2 + static_cast<size_t>(TB) * a.E * 4 * (a.mode == 1 ? 2 : 1);
-  if (a.fuse_permute) {
-    const size_t need = static_cast<size_t>(kRouterThreads / 32 + 2) * a.E * 4 + 4;
+  if (a.fuse_permute) {  // permute_body's wc, cnt, base over all experts (shared included)
+    const size_t need = static_cast<size_t>(kRouterThreads / 32 + 2) * a.perm.E * 4 + 4;
     smem = smem > need ? smem : need;
   }
   cudaError_t err = set_max_dynamic_smem<router_kernel<TB, EG>>(160 * 1024);

@@ -31,7 +31,7 @@ def test_header_symbols_are_exported():
 
 
 def test_abi_version_and_strings():
-    assert capi.abi_version() == 2
+    assert capi.abi_version() == 3
     for code, name in [(0, "FMOE_OK"), (1, "FMOE_ERR_INVALID_ARG"), (2, "FMOE_ERR_UNSUPPORTED"),
                        (3, "FMOE_ERR_WORKSPACE"), (4, "FMOE_ERR_CUDA"), (5, "FMOE_ERR_TIMEOUT"),
                        (6, "FMOE_ERR_DEVICE_BOUNDS")]:
@@ -125,6 +125,25 @@ def test_launch_counts():
     # the CTA-pair kernels launch once per contraction like the one-CTA ones
     assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal_pair")) == 5
     assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2, variant="normal_pair")) == 7
+
+
+def test_shared_expert_validation_and_workspace():
+    # n_shared outside 0..8 is rejected; shared experts add K = k + S slots per token
+    for bad in (-1, 9):
+        d = dims()
+        r = capi.make_softmax_routing(bad)
+        d = capi.make_dims(4, 256, 512, 8, 2, True, routing=r)
+        assert call_fused(d) == capi.FMOE_ERR_INVALID_ARG
+    base = capi.workspace_size(dims(T=64, H=4096, I=1024))
+    r = capi.make_softmax_routing(1)
+    with_shared = capi.workspace_size(capi.make_dims(64, 4096, 1024, 8, 2, True, routing=r))
+    assert with_shared > base
+    # same launch sequence with or without shared experts
+    assert capi.fused_moe_launches_per_call(capi.make_dims(4, 256, 512, 8, 2, True, "swap_ab",
+                                                           routing=r)) == 6
+    # E + S may exceed 256 (DeepSeek-V3: 256 routed + 1 shared)
+    g = capi.make_routing(8, 4, 2.5, None, n_shared=1)
+    assert capi.workspace_size(capi.make_dims(16, 7168, 2048, 256, 8, True, routing=g)) > 0
 
 
 def test_variant_choice_and_pair_workspace():

@@ -36,10 +36,12 @@ def dev_inputs(inp: minp.MoEInputs):
 
 
 def routing_of(inp):
-    if inp.shape.grouped is None:
-        return None
-    n_group, topk_group, scaling = inp.shape.grouped
-    return capi.make_routing(n_group, topk_group, scaling, inp.router_bias.cuda())
+    s = inp.shape
+    if s.grouped is None:
+        return capi.make_softmax_routing(s.n_shared) if s.n_shared else None
+    n_group, topk_group, scaling = s.grouped
+    return capi.make_routing(n_group, topk_group, scaling, inp.router_bias.cuda(),
+                             n_shared=s.n_shared)
 
 
 def bits16(t: torch.Tensor) -> np.ndarray:
@@ -55,8 +57,8 @@ def run_steps(inp, g, variant="auto", a1=0.0, a2=0.0):
     dev = "cuda"
     ids = torch.empty(R, dtype=torch.int32, device=dev)
     tw = torch.empty(R, dtype=torch.float32, device=dev)
-    counts = torch.empty(s.E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(s.E + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(s.E_all, dtype=torch.int32, device=dev)
+    offsets = torch.empty(s.E_all + 1, dtype=torch.int32, device=dev)
     rows = torch.empty(R, dtype=torch.int32, device=dev)
     inv = torch.empty(R, dtype=torch.int32, device=dev)
     a_perm = torch.empty(R, s.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
@@ -70,8 +72,9 @@ def run_steps(inp, g, variant="auto", a1=0.0, a2=0.0):
     torch.cuda.synchronize()
     assert capi.fused_moe_get_device_status(ws) == capi.FMOE_OK
     fs, ints = capi.fused_moe_debug_scalars(ws)
-    return dict(topk_ids=ids.cpu().numpy().reshape(s.T, s.top_k),
-                topk_w=tw.cpu().numpy().reshape(s.T, s.top_k),
+    K = s.top_k + s.n_shared  # slots per token: routed, then shared
+    return dict(topk_ids=ids.cpu().numpy().reshape(s.T, K),
+                topk_w=tw.cpu().numpy().reshape(s.T, K),
                 counts=counts.cpu().numpy(), offsets=offsets.cpu().numpy(),
                 sorted_rows=rows.cpu().numpy(), inv_perm=inv.cpu().numpy(),
                 a_perm=a_perm.cpu().numpy() if fp8 else bits16(a_perm),
@@ -133,6 +136,12 @@ SMALL = [
     # more than 256 rows per expert: several CTA-pair chunks with ragged tails
     ("fp8_pair_chunks", (700, 512, 384, 2, 1, "fp8"), {}),
     ("bf16_pair_chunks", (600, 256, 256, 3, 2, "bf16"), {}),
+    # shared experts (every token, weight 1, after the routed slots)
+    ("fp8_shared", (37, 512, 384, 8, 2, "fp8"), {"n_shared": 1}),
+    ("bf16_shared_two", (21, 256, 256, 6, 2, "bf16"), {"n_shared": 2}),
+    ("fp8_grouped_shared", (64, 512, 256, 64, 8, "fp8"),
+     {"router_std": 1.0, "grouped": (8, 4, 2.5), "n_shared": 1}),
+    ("fp8_shared_pair_chunks", (300, 256, 256, 4, 2, "fp8"), {"n_shared": 1}),
 ]
 
 
@@ -183,7 +192,7 @@ def test_small_fused_equals_steps_and_variants_agree(small_cases, name):
 
 
 @pytest.mark.parametrize("name", ["tiny_bf16", "fp8_ragged", "fp8_multichunk", "fp8_pair_chunks",
-                                  "bf16_pair_chunks", "fp8_many_experts"])
+                                  "bf16_pair_chunks", "fp8_many_experts", "fp8_shared_pair_chunks"])
 def test_pair_variant_equals_normal(small_cases, name):
     """The CTA-pair kernel runs the normal variant's tiles with the same K order and the
     same epilogue arithmetic: identical output bits."""
@@ -304,19 +313,23 @@ def test_router_full_shapes(workload, T):
     routing = None
     if s.grouped is None:
         ids_ref, w_ref, _ = O.router(minp.bf16_bits(x), minp.bf16_bits(wr), s.top_k)
+        if s.n_shared:
+            routing = capi.make_softmax_routing(s.n_shared)
     else:
         bias = minp.make_router_bias(s, seed=0)
         ids_ref, w_ref, _, _ = O.router_grouped(
             minp.bf16_bits(x), minp.bf16_bits(wr), s.top_k, n_group=s.grouped[0],
             topk_group=s.grouped[1], routed_scaling=s.grouped[2], bias=bias.numpy())
-        routing = capi.make_routing(*s.grouped, bias.cuda())
-    counts_ref, offs_ref, rows_ref, inv_ref = O.permute(ids_ref, s.E)
+        routing = capi.make_routing(*s.grouped, bias.cuda(), n_shared=s.n_shared)
+    ids_ref, w_ref = O.append_shared(ids_ref, w_ref, s.E, s.n_shared)
+    counts_ref, offs_ref, rows_ref, inv_ref = O.permute(ids_ref, s.E_all)
     dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, True, routing=routing)
     ws = capi.alloc_workspace(dims)
     R = s.R
+    K = s.top_k + s.n_shared
     ids = torch.empty(R, dtype=torch.int32, device="cuda")
     tw = torch.empty(R, dtype=torch.float32, device="cuda")
-    bufs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (s.E, s.E + 1, R, R)]
+    bufs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (s.E_all, s.E_all + 1, R, R)]
     a_perm = torch.empty(R, s.H, dtype=torch.uint8, device="cuda")
     xd = x.cuda()
     for _ in range(2):  # the second call starts from the counters the first one left
@@ -324,8 +337,8 @@ def test_router_full_shapes(workload, T):
         capi.fused_moe_permute(dims, ids, xd, None, *bufs, a_perm, ws)
         torch.cuda.synchronize()
         assert capi.fused_moe_get_device_status(ws) == capi.FMOE_OK
-        assert np.array_equal(ids.cpu().numpy().reshape(s.T, s.top_k), ids_ref)
-        assert np.allclose(tw.cpu().numpy().reshape(s.T, s.top_k), w_ref, rtol=1e-6, atol=1e-9)
+        assert np.array_equal(ids.cpu().numpy().reshape(s.T, K), ids_ref)
+        assert np.allclose(tw.cpu().numpy().reshape(s.T, K), w_ref, rtol=1e-6, atol=1e-9)
         for got, ref in zip(bufs, (counts_ref, offs_ref, rows_ref, inv_ref)):
             assert np.array_equal(got.cpu().numpy(), ref)
 
@@ -333,7 +346,8 @@ def test_router_full_shapes(workload, T):
 @pytest.mark.parametrize("name,variant", [("fp8_ragged", "swap_ab"), ("fp8_multichunk", "normal"),
                                           ("bf16_multichunk", "swap_ab"),
                                           ("fp8_pair_chunks", "normal_pair"),
-                                          ("bf16_pair_chunks", "normal_pair")])
+                                          ("bf16_pair_chunks", "normal_pair"),
+                                          ("fp8_grouped_shared", "swap_ab")])
 def test_poisoned_workspace_and_outputs_are_fully_rewritten(small_cases, name, variant):
     """Workspace (apart from its initialised header) and every output start as NaN
     bytes: a kernel that read a region it had not written, or left an output element
@@ -341,7 +355,7 @@ def test_poisoned_workspace_and_outputs_are_fully_rewritten(small_cases, name, v
     inp, g, ref = small_cases(name)
     s = inp.shape
     fp8 = s.wdtype == "fp8"
-    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, variant)
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, variant, routing=g.get("routing"))
     ws = capi.alloc_workspace(dims)
     ws.fill_(0xFF)
     capi.fused_moe_workspace_init(ws)
