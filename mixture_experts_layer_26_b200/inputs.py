@@ -172,3 +172,57 @@ def make_inputs(s: MoEShape, seed: int = 0) -> MoEInputs:
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a bf16 tensor's bits."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+# ------------------------------------------------------------------------------------
+# Inputs of the inverse-rotary + per-head FP8 quantisation kernel
+# ------------------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class RopeShape:
+    T: int          # tokens
+    n_heads: int
+    head_dim: int
+    rot_dim: int    # rotated leading coordinates of each head (even, <= head_dim)
+    style: int = 0  # 0: pairs (i, i + rot_dim/2); 1: pairs (2i, 2i+1)
+    max_pos: int = 32768
+    base: float = 10000.0
+    name: str = ""
+
+
+# A prefill batch of Mixtral-like attention (32 query heads of 128) on one GPU, the
+# same with 8-way tensor parallelism (4 heads per GPU), and a partial-rotary
+# interleaved layout.
+ROPE_WORKLOADS = {
+    "inv_rope_fp8_prefill": dict(T=16384, n_heads=32, head_dim=128, rot_dim=128),
+    "inv_rope_fp8_tp8": dict(T=16384, n_heads=4, head_dim=128, rot_dim=128),
+    "inv_rope_fp8_partial": dict(T=4096, n_heads=16, head_dim=128, rot_dim=64, style=1),
+}
+
+
+def rope_shape(workload: str, T: Optional[int] = None) -> RopeShape:
+    w = dict(ROPE_WORKLOADS[workload])
+    if T is not None:
+        w["T"] = T
+    return RopeShape(name=workload, **w)
+
+
+@dataclasses.dataclass
+class RopeInputs:
+    shape: RopeShape
+    x: torch.Tensor          # [T, n_heads, head_dim] bf16
+    positions: torch.Tensor  # [T] int32
+    cos_sin: torch.Tensor    # [max_pos, rot_dim] fp32: rot_dim/2 cosines, then sines
+
+
+def make_rope_inputs(s: RopeShape, seed: int = 0) -> RopeInputs:
+    """x ~ N(0, 1) in bf16; positions drawn uniformly from [0, max_pos); the rotary table
+    of a model with the given base: angle(p, i) = p * base^(-2i/rot_dim), evaluated in
+    fp64 and stored as fp32 cosines and sines (a cache the model keeps)."""
+    x = torch.randn(s.T, s.n_heads, s.head_dim, generator=_gen(seed, 11), dtype=torch.float32)
+    pos = torch.randint(0, s.max_pos, (s.T,), generator=_gen(seed, 12), dtype=torch.int64)
+    half = s.rot_dim // 2
+    inv_freq = s.base ** (-torch.arange(half, dtype=torch.float64) * 2.0 / s.rot_dim)
+    ang = torch.arange(s.max_pos, dtype=torch.float64)[:, None] * inv_freq[None, :]
+    table = torch.cat([ang.cos(), ang.sin()], dim=1).to(torch.float32).contiguous()
+    return RopeInputs(s, x.to(torch.bfloat16), pos.to(torch.int32), table)
