@@ -71,7 +71,9 @@ def load_peaks():
 
 def gemm_source_hash(kernel: str = "") -> str:
     h = hashlib.sha256()
-    for rel in (PAIR_GEMM_SOURCES if "pair" in kernel else GEMM_SOURCES):
+    srcs = ROPE_SOURCES if "rope" in kernel else (PAIR_GEMM_SOURCES if "pair" in kernel
+                                                   else GEMM_SOURCES)
+    for rel in srcs:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -474,14 +476,204 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+# --------------------------------------------------------------------------- inverse RoPE
+
+ROPE_METRIC = ("inverse-RoPE + per-head FP8 quantisation tokens/s; achieved HBM GB/s vs peak")
+ROPE_SOURCES = ("mixture_experts_layer_26_b200/csrc/inv_rope_fp8.cu",
+                "mixture_experts_layer_26_b200/csrc/fmoe_common.cuh")
+
+
+def rope_bytes(s) -> int:
+    """Algorithmic bytes of one launch: x read (bf16), codes written, scales written,
+    positions read, and the rotary table rows the tokens gather (rot_dim fp32 each)."""
+    el = s.T * s.n_heads * s.head_dim
+    return el * 2 + el + s.T * s.n_heads * 4 + s.T * 4 + s.T * s.rot_dim * 4
+
+
+def rope_config(s):
+    x_bytes = s.T * s.n_heads * s.head_dim * 2
+    big = x_bytes > L2_BYTES
+    return {"workload": f"{s.name}: T={s.T} heads={s.n_heads} head_dim={s.head_dim} "
+                        f"rot_dim={s.rot_dim} style={'half-split' if s.style == 0 else 'interleaved'}",
+            "T": s.T, "n_heads": s.n_heads, "head_dim": s.head_dim, "rot_dim": s.rot_dim,
+            "style": s.style, "max_pos": s.max_pos,
+            "l2": (f"inputs larger than L2 ({x_bytes / 2 ** 20:.0f} MB x), no flush" if big else
+                   f"L2 flushed before every timed launch ({x_bytes / 2 ** 20:.0f} MB x < "
+                   f"{L2_BYTES / 2 ** 20:.0f} MB L2)"),
+            "parallelism": "replicas (one independent kernel per GPU)"}
+
+
+def rope_oracle_seconds(inp, tokens):
+    """The oracle on the first `tokens` tokens of the batch: seconds."""
+    from oracle import inv_rope_fp8_oracle as RO
+    s = inp.shape
+    xb = inp.x[:tokens].contiguous().view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    RO.inv_rope_fp8_quant(xb, inp.positions[:tokens].numpy(), inp.cos_sin.numpy(), s.rot_dim,
+                          s.style)
+    return time.perf_counter() - t0
+
+
+def run_rope_ours(args, rank, world, local_rank):
+    from mixture_experts_layer_26_b200 import capi
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = minp.rope_shape(args.workload, args.T)
+    inp = minp.make_rope_inputs(s, seed=0)
+    x, pos, cs = inp.x.to(dev), inp.positions.to(dev), inp.cos_sin.to(dev)
+    q = torch.empty(s.T, s.n_heads, s.head_dim, dtype=torch.uint8, device=dev)
+    sc = torch.empty(s.T, s.n_heads, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    d = capi.make_rope_dims(s.T, s.n_heads, s.head_dim, s.rot_dim, s.style, s.max_pos)
+    stream = torch.cuda.current_stream(dev)
+    flush = s.T * s.n_heads * s.head_dim * 2 <= L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def launch():
+        capi.fused_inv_rope_fp8_quant_per_head(d, x, pos, cs, q, sc, status, stream)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    assert int(status.item()) == capi.FMOE_OK
+
+    # ---- timed region: exactly K launches; with small inputs the L2 is flushed before
+    # each launch and only the launches are timed (events around each one)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev)) if rank == 0 else None
+    if flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for e0, e1 in evs:
+            scratch.fill_(1)
+            e0.record(stream)
+            launch()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            launch()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+    barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    ms = reduce_max(dist, ms, dev)
+    assert int(status.item()) == capi.FMOE_OK
+    ms_launch = ms / args.steps
+    value = tokens_per_second(world, s.T, args.steps, ms)
+
+    # ---- end to end: x and positions from pinned host memory, codes and scales back
+    x_h, pos_h = inp.x.clone().pin_memory(), inp.positions.clone().pin_memory()
+    q_h = torch.empty(q.shape, dtype=torch.uint8).pin_memory()
+    sc_h = torch.empty(sc.shape, dtype=torch.float32).pin_memory()
+    n_e2e = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        pos.copy_(pos_h, non_blocking=True)
+        launch()
+        q_h.copy_(q, non_blocking=True)
+        sc_h.copy_(sc, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(dist, a0.elapsed_time(a1), dev)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    nbytes = rope_bytes(s)
+    ach = nbytes / (ms_launch / 1e3) / 1e9
+    kname = "inv_rope_fp8"
+    roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4),
+            "traffic": profiled_traffic(kname, f"{args.workload}_T{s.T}"),
+            "kernel": kname, "kernel_us": round(1e3 * ms_launch, 2), "algorithmic_bytes": nbytes,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n = min(s.T, 2048)
+        secs = rope_oracle_seconds(inp, n)
+        cpu = {"value": n / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"the oracle on the first {n} of the {s.T} tokens ({secs:.2f} s)"}
+    el = s.T * s.n_heads * s.head_dim
+    line = {
+        "metric": ROPE_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_launch, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in, fp32 rotation, e4m3 + fp32 per-head scales out",
+        "data": "synthetic (seeded; N(0,1) x, uniform positions, rotary table of base 10000)",
+        "config": rope_config(s), "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": round(tokens_per_second(world, s.T, n_e2e, e2e_ms), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": el * 2 + s.T * 4,
+                "d2h_bytes_per_step": el + s.T * s.n_heads * 4,
+                "api": "fused_inv_rope_fp8_quant_per_head with pinned host copies"},
+        "gpu_launches": args.steps, "clocks": clocks,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_rope_reference(args, rank):
+    if rank != 0:
+        return 0
+    s = minp.rope_shape(args.workload, args.T)
+    inp = minp.make_rope_inputs(s, seed=0)
+    n = min(s.T, 1024)  # each step: the oracle on a bounded slice of the batch
+    for _ in range(min(args.warmup, 2)):
+        rope_oracle_seconds(inp, n)
+    total = sum(rope_oracle_seconds(inp, n) for _ in range(args.steps))
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": ROPE_METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32 (oracle)", "data": "synthetic",
+        "config": rope_config(s),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": f"{args.steps} steps of {n} tokens each"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral_fp8_decode", choices=sorted(minp.WORKLOADS))
-    ap.add_argument("--T", type=int, default=64)
+    ap.add_argument("--workload", default="mixtral_fp8_decode",
+                    choices=sorted(minp.WORKLOADS) + sorted(minp.ROPE_WORKLOADS))
+    ap.add_argument("--T", type=int, default=None,
+                    help="tokens (default: the workload's largest; 64 for the default workload)")
     ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal", "normal_pair"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -490,6 +682,10 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in minp.ROPE_WORKLOADS:
+        if args.impl == "reference":
+            return run_rope_reference(args, rank)
+        return run_rope_ours(args, rank, world, local_rank)
     if args.impl == "reference":
         return run_reference(args, rank)
     return run_ours(args, rank, world, local_rank)

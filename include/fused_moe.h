@@ -251,6 +251,52 @@ FMOE_API fmoe_status fused_moe_profile(const fmoe_dims* dims, const void* x, con
                                        float* ms_host, const char** names_host, int32_t cap,
                                        int32_t* n_host);
 
+/* ---------------------------------------------------------------------------------
+ * Fused inverse rotary embedding + per-head FP8 quantisation.
+ *
+ * The pages' second kernel: a fused rotary-embedding plus FP8-quantisation kernel
+ * (`_fused_inv_rope_fp8_quant_per_head`) that Triton recompiled for every new token
+ * count (codebridge-ai.com blog "AWS MoE kernel: WGMMA, Triton, TTFT", section "3. Kill
+ * JIT recompilation"; agentic-affairs.com, third change).  The pages give no formula;
+ * this is the plainest reading of the name.  Token t of x was rotated by the angles of
+ * its position pos[t]; the call undoes that and quantises every head:
+ *   pairs (a, b) of the first rot_dim coordinates of a head, (i, i + rot_dim/2) for
+ *   style 0 (half split) or (2i, 2i+1) for style 1 (interleaved), i < rot_dim/2:
+ *     y_a =  x_a * cos(pos, i) + x_b * sin(pos, i)
+ *     y_b = -(x_a * sin(pos, i)) + x_b * cos(pos, i)
+ *   each product and each sum rounded to fp32 separately (no fused multiply-add);
+ *   coordinates rot_dim..head_dim-1 pass through (y = x);
+ *   scales[t, h] = max|y| / 448 over the head (1 for an all-zero head) and
+ *   q = e4m3(y * (448 / max|y|)), the product in fp32, round to nearest even,
+ *   saturating to +-448.
+ */
+typedef struct {
+  int32_t T;         /* tokens (0: nothing to do) */
+  int32_t n_heads;   /* >= 1 */
+  int32_t head_dim;  /* 64, 128 or 256 */
+  int32_t rot_dim;   /* rotated coordinates per head: 2*head_dim/32 <= rot_dim <= head_dim;
+                        style 0: a power of two; style 1: a multiple of 2*head_dim/32 */
+  int32_t style;     /* 0: pairs (i, i + rot_dim/2); 1: pairs (2i, 2i+1) */
+  int32_t max_pos;   /* rows of the rotary table, >= 1 */
+} fmoe_rope_dims;
+
+/* x         [T, n_heads, head_dim] bf16, device
+ * positions [T] int32, device: row of cos_sin for each token; a position outside
+ *           [0, max_pos) is treated as 0 and reported as FMOE_ERR_DEVICE_BOUNDS in
+ *           *device_status (if not NULL)
+ * cos_sin   [max_pos, rot_dim] fp32, device: the rot_dim/2 cosines, then the rot_dim/2
+ *           sines of each position's angles
+ * q         [T, n_heads, head_dim] e4m3 bytes out, device
+ * scales    [T, n_heads] fp32 out, device
+ * device_status  int32 device word or NULL; first error kept (set it to 0 beforehand)
+ * All device pointers 16-byte aligned.  Asynchronous on `stream`; no workspace.
+ * Errors: FMOE_ERR_INVALID_ARG (null pointer, sizes outside the ranges above),
+ * FMOE_ERR_UNSUPPORTED (alignment, element counts >= 2^31), FMOE_ERR_CUDA. */
+FMOE_API fmoe_status fused_inv_rope_fp8_quant_per_head(const fmoe_rope_dims* dims, const void* x,
+                                                       const int32_t* positions, const float* cos_sin,
+                                                       void* q, float* scales, int32_t* device_status,
+                                                       fmoe_stream stream);
+
 /* Size of the library-owned workspace used by fused_moe_static_workspace: 64 MiB. */
 #define FUSED_MOE_STATIC_WS_BYTES ((size_t)64 << 20)
 

@@ -37,6 +37,7 @@ EXPORTED = (
     "fused_moe_combine", "fused_moe", "fused_moe_host_io", "fused_moe_get_device_status",
     "fused_moe_debug_scalars", "fused_moe_launches_per_call", "fused_moe_profile",
     "fused_moe_static_workspace", "fused_moe_selftest_wait",
+    "fused_inv_rope_fp8_quant_per_head",
 )
 STATIC_WS_BYTES = 64 << 20  # FUSED_MOE_STATIC_WS_BYTES
 
@@ -53,6 +54,11 @@ class FmoeDims(ctypes.Structure):
     _fields_ = [("T", c_int32), ("H", c_int32), ("I", c_int32), ("E", c_int32),
                 ("top_k", c_int32), ("wdtype", c_int32), ("variant", c_int32),
                 ("routing", POINTER(FmoeRouting))]
+
+
+class FmoeRopeDims(ctypes.Structure):
+    _fields_ = [("T", c_int32), ("n_heads", c_int32), ("head_dim", c_int32),
+                ("rot_dim", c_int32), ("style", c_int32), ("max_pos", c_int32)]
 
 
 class FmoeScales(ctypes.Structure):
@@ -92,6 +98,8 @@ _selftest_wait = _sig("fused_moe_selftest_wait", c_int32, c_void_p, c_size_t, ct
                       c_void_p)
 _static_ws = _sig("fused_moe_static_workspace", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p,
                   _SP, c_void_p, c_void_p, c_void_p)
+_inv_rope = _sig("fused_inv_rope_fp8_quant_per_head", c_int32, POINTER(FmoeRopeDims), c_void_p,
+                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p)
 _profile = _sig("fused_moe_profile", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
                 c_void_p, c_void_p, c_size_t, c_void_p, POINTER(c_float), POINTER(c_char_p),
                 c_int32, POINTER(c_int32))
@@ -310,3 +318,17 @@ class FusedMoE:
         fused_moe(self.dims(T), x, self.router_w, self.w13, self.w2, self.scales, out,
                   self.workspace(T), stream)
         return out
+
+
+def make_rope_dims(T: int, n_heads: int, head_dim: int, rot_dim: int, style: int = 0,
+                   max_pos: int = 32768) -> FmoeRopeDims:
+    return FmoeRopeDims(T, n_heads, head_dim, rot_dim, style, max_pos)
+
+
+def fused_inv_rope_fp8_quant_per_head(dims: FmoeRopeDims, x, positions, cos_sin, q, scales,
+                                      device_status=None, stream=None, check=True) -> int:
+    """x [T,n_heads,head_dim] bf16, positions [T] int32, cos_sin [max_pos,rot_dim] fp32 ->
+    q [T,n_heads,head_dim] uint8 (e4m3 codes), scales [T,n_heads] fp32 (device tensors)."""
+    st = _inv_rope(ctypes.byref(dims), _ptr(x), _ptr(positions), _ptr(cos_sin), _ptr(q),
+                   _ptr(scales), _ptr(device_status), _stream(stream))
+    return _check(st, "fused_inv_rope_fp8_quant_per_head") if check else st

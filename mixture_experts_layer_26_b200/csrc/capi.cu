@@ -760,4 +760,39 @@ fmoe_status fused_moe_debug_scalars(const void* ws, float* f6, int32_t* i3, fmoe
   return FMOE_OK;
 }
 
+fmoe_status fused_inv_rope_fp8_quant_per_head(const fmoe_rope_dims* d, const void* x,
+                                              const int32_t* positions, const float* cos_sin,
+                                              void* q, float* scales, int32_t* device_status,
+                                              fmoe_stream stream) {
+  if (d == nullptr) return FMOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->n_heads < 1 || d->max_pos < 1 || (d->style != 0 && d->style != 1))
+    return FMOE_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return FMOE_ERR_INVALID_ARG;
+  const int epl = d->head_dim / 32, r = d->rot_dim;
+  if (r < 2 * epl || r > d->head_dim) return FMOE_ERR_INVALID_ARG;
+  if (d->style == 0 ? (r & (r - 1)) != 0 : r % (2 * epl) != 0) return FMOE_ERR_INVALID_ARG;
+  const int64_t lim = int64_t(1) << 31;
+  if (static_cast<int64_t>(d->T) * d->n_heads * d->head_dim >= lim ||
+      static_cast<int64_t>(d->max_pos) * r >= lim)
+    return FMOE_ERR_UNSUPPORTED;
+  if (d->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, positions, cos_sin, q, scales));
+  if (device_status != nullptr && (reinterpret_cast<uintptr_t>(device_status) & 3u) != 0)
+    return FMOE_ERR_UNSUPPORTED;
+  RopeArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.positions = positions;
+  a.cos_sin = cos_sin;
+  a.q = static_cast<uint8_t*>(q);
+  a.scales = scales;
+  a.status = device_status;
+  a.T = d->T;
+  a.n_heads = d->n_heads;
+  a.head_dim = d->head_dim;
+  a.rot_dim = r;
+  a.style = d->style;
+  a.max_pos = d->max_pos;
+  return cuda_status(launch_inv_rope_fp8(a, num_sms(), static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

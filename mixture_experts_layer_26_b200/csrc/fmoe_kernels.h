@@ -220,4 +220,17 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
 
+// ----------------------------------------------------------------------------- inverse RoPE
+struct RopeArgs {
+  const uint16_t* x;        // [T, n_heads, head_dim] bf16
+  const int32_t* positions; // [T]
+  const float* cos_sin;     // [max_pos, rot_dim]: rot_dim/2 cosines, then sines
+  uint8_t* q;               // [T, n_heads, head_dim] e4m3
+  float* scales;            // [T, n_heads]
+  int32_t* status;          // device status word (FMOE_ERR_DEVICE_BOUNDS), or null
+  int T, n_heads, head_dim, rot_dim, style, max_pos;
+};
+// head_dim in {64, 128, 256}; rot_dim checked by the caller (see fused_moe.h).
+cudaError_t launch_inv_rope_fp8(const RopeArgs& a, int num_sms, cudaStream_t s);
+
 }  // namespace fmoe

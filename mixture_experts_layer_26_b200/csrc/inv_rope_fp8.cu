@@ -1,0 +1,252 @@
+// Fused inverse rotary embedding + per-head FP8 quantisation.
+//
+// The second kernel the pages optimise: a fused rotary-embedding plus FP8-quantisation
+// kernel that Triton recompiled for every new token count (codebridge-ai.com blog "AWS
+// MoE kernel: WGMMA, Triton, TTFT", section "3. Kill JIT recompilation";
+// agentic-affairs.com, third change).  This one is compiled ahead of time for every
+// shape, so the recompilation the pages fix cannot arise.
+//
+// For token t (position pos[t]) and head h of x [T, n_heads, head_dim] (bf16):
+//   pairs (a, b) of the first rot_dim coordinates, (i, i + rot_dim/2) (style 0) or
+//   (2i, 2i+1) (style 1), are rotated by -theta(pos, i):
+//     y_a = x_a*cos + x_b*sin,  y_b = -(x_a*sin) + x_b*cos
+//   each product and each sum rounded to fp32 separately (no fused multiply-add), in
+//   that order; coordinates past rot_dim pass through;
+//   scale[t, h] = amax|y| / 448 (1 if the head is zero), q = e4m3(y * (448/amax)),
+//   round to nearest even, saturating.
+//
+// HBM-bound: 2 bytes read and 1 byte written per element plus 4 bytes of scale per
+// head; the rotary table (max_pos x rot_dim fp32) is gathered through L2.  One warp
+// handles up to eight heads of one token per step, lane l owning the EPL = head_dim/32
+// consecutive coordinates [EPL*l, EPL*l + EPL) of each head: one vector load and one
+// packed store per head and lane, with the next step's loads in flight meanwhile.  The
+// half-split partner of a coordinate lives rot_dim/(2*EPL) lanes away (a lane xor for
+// power-of-two rot_dim); interleaved partners are in the same lane.  The grid is the
+// number of blocks that fit on the GPU at once (a persistent grid-stride loop).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "fmoe_kernels.h"
+
+namespace fmoe {
+
+namespace {
+
+constexpr int kRopeThreads = 256;
+
+template <int EPL> struct Vec;
+template <> struct Vec<2> { using X = uint32_t; using F = float2; using Q = uint16_t; };
+template <> struct Vec<4> { using X = uint2; using F = float4; using Q = uint32_t; };
+template <> struct Vec<8> { using X = uint4; using F = float4; using Q = uint2; };
+
+template <int EPL>
+__device__ __forceinline__ void unpack_bf16(const typename Vec<EPL>::X& v, float (&f)[EPL]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+  for (int i = 0; i < EPL / 2; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// n consecutive fp32 values of a table row (n = 1, 2, 4 or 8; 4-byte aligned at least
+// n*4 bytes when n <= 4, 16 bytes when n == 8).
+template <int N>
+__device__ __forceinline__ void load_row(const float* p, float (&v)[N]) {
+  if constexpr (N == 1) {
+    v[0] = __ldg(p);
+  } else if constexpr (N == 2) {
+    const float2 a = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = a.x; v[1] = a.y;
+  } else if constexpr (N == 4) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// Heads a warp takes per step: 8 (4 for head_dim 256), so that each lane keeps 32 bytes
+// of x per step.
+template <int EPL> constexpr int heads_per_step() { return EPL == 8 ? 4 : 8; }
+
+template <int EPL, int kStyle>
+__global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int HPS = heads_per_step<EPL>();
+  constexpr int NC = kStyle == 0 ? EPL : EPL / 2;  // table entries a lane needs
+  constexpr int NW = EPL / 2;                      // 32-bit words (bf16 pairs) per lane
+  using XV = typename Vec<EPL>::X;
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * kRopeThreads + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * kRopeThreads) >> 5;
+  const int hd = 32 * EPL, rot = a.rot_dim, half = rot / 2;
+  const int j0 = lane * EPL;               // first coordinate of this lane
+  const bool rotated = j0 < rot;           // EPL divides rot: a lane is all in or all out
+  const bool is_a = kStyle == 0 ? j0 < half : true;
+  // style 0: pair index of coordinate j0 (its partner's too); style 1: j0 / 2
+  const int i0 = kStyle == 0 ? (is_a ? j0 : j0 - half) : j0 / 2;
+  const int partner_xor = kStyle == 0 ? half / EPL : 0;
+  const int hgroups = (a.n_heads + HPS - 1) / HPS;
+  const int units = a.T * hgroups;  // < 2^31: T * n_heads * head_dim is checked on the host
+
+  // Software pipeline over this warp's units u, u + nwarps, ...: the position of unit
+  // u + 2*nwarps and the x rows and table entries of unit u + nwarps are in flight while
+  // unit u is rotated, quantised and stored.
+  struct Unit {
+    int t, h0;
+  };
+  auto unit_of = [&](int u) { return Unit{u / hgroups, (u % hgroups) * HPS}; };
+  auto pos_of = [&](int u) -> int {
+    if (u >= units) return 0;
+    const Unit w = unit_of(u);
+    int p = __ldg(a.positions + w.t);
+    if (p < 0 || p >= a.max_pos) {
+      if (lane == 0 && w.h0 == 0 && a.status != nullptr) record_status(a.status, ST_BOUNDS);
+      p = 0;
+    }
+    return p;
+  };
+  auto load_x = [&](int u, XV (&xv)[HPS]) {
+    if (u >= units) return;
+    const Unit w = unit_of(u);
+    const XV* src = reinterpret_cast<const XV*>(
+        a.x + (static_cast<size_t>(w.t) * a.n_heads + w.h0) * hd + j0);
+#pragma unroll
+    for (int k = 0; k < HPS; ++k)
+      if (w.h0 + k < a.n_heads) xv[k] = __ldcs(src + k * 32);  // streamed once
+  };
+  auto load_table = [&](int u, int p, float (&cs)[NC], float (&sn)[NC]) {
+    if (u >= units || !rotated) return;
+    const float* row = a.cos_sin + static_cast<size_t>(p) * rot;
+    load_row<NC>(row + i0, cs);
+    load_row<NC>(row + half + i0, sn);
+  };
+
+  int u = gwarp;
+  XV xc[HPS], xn[HPS];
+  float cc[NC], sc_[NC], cn[NC], sn_[NC];
+  int p_next = pos_of(u + nwarps);
+  {
+    const int p0 = pos_of(u);
+    load_x(u, xc);
+    load_table(u, p0, cc, sc_);
+  }
+  for (; u < units; u += nwarps) {
+    // next unit's x and table (its position is already here), the one after's position
+    load_x(u + nwarps, xn);
+    load_table(u + nwarps, p_next, cn, sn_);
+    const int p_after = pos_of(u + 2 * nwarps);
+
+    const Unit w = unit_of(u);
+    uint8_t* qdst = a.q + (static_cast<size_t>(w.t) * a.n_heads + w.h0) * hd + j0;
+    float* sdst = a.scales + static_cast<size_t>(w.t) * a.n_heads + w.h0;
+#pragma unroll
+    for (int k = 0; k < HPS; ++k) {
+      if (w.h0 + k >= a.n_heads) break;  // warp-uniform
+      float x[EPL], y[EPL];
+      unpack_bf16<EPL>(xc[k], x);
+      if constexpr (kStyle == 0) {
+        // the partner's coordinates, moved as packed bf16 pairs (one shuffle per word)
+        const uint32_t* wv = reinterpret_cast<const uint32_t*>(&xc[k]);
+        float o[EPL];
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+          const uint32_t ow = __shfl_xor_sync(0xffffffffu, wv[i], partner_xor);
+          o[2 * i] = __uint_as_float(ow << 16);
+          o[2 * i + 1] = __uint_as_float(ow & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          if (!rotated) {
+            y[e] = x[e];
+          } else if (is_a) {  // x[e] = x_a, o = x_b
+            y[e] = __fadd_rn(__fmul_rn(x[e], cc[e]), __fmul_rn(o[e], sc_[e]));
+          } else {            // x[e] = x_b, o = x_a
+            y[e] = __fadd_rn(-__fmul_rn(o[e], sc_[e]), __fmul_rn(x[e], cc[e]));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; e += 2) {
+          if (!rotated) {
+            y[e] = x[e];
+            y[e + 1] = x[e + 1];
+          } else {
+            const float c = cc[e / 2], s = sc_[e / 2];
+            y[e] = __fadd_rn(__fmul_rn(x[e], c), __fmul_rn(x[e + 1], s));
+            y[e + 1] = __fadd_rn(-__fmul_rn(x[e], s), __fmul_rn(x[e + 1], c));
+          }
+        }
+      }
+      // max |y| over the head: the bit patterns of non-negative finite floats order like
+      // unsigned integers, so one warp-wide unsigned max gives it exactly
+      uint32_t mb = 0;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) mb = max(mb, __float_as_uint(y[e]) & 0x7FFFFFFFu);
+      const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, mb));
+      const float inv = m > 0.f ? 448.0f / m : 1.f;
+      typename Vec<EPL>::Q qv;
+      uint16_t* q16 = reinterpret_cast<uint16_t*>(&qv);
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2)
+        q16[e / 2] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(
+            make_float2(__fmul_rn(y[e], inv), __fmul_rn(y[e + 1], inv)), __NV_SATFINITE, __NV_E4M3));
+      __stcs(reinterpret_cast<typename Vec<EPL>::Q*>(qdst + k * hd), qv);
+      if (lane == 0) __stcs(sdst + k, m > 0.f ? m / 448.0f : 1.f);
+    }
+#pragma unroll
+    for (int k = 0; k < HPS; ++k) xc[k] = xn[k];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      cc[i] = cn[i];
+      sc_[i] = sn_[i];
+    }
+    p_next = p_after;
+  }
+}
+
+template <int EPL, int kStyle>
+cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
+  constexpr int HPS = heads_per_step<EPL>();
+  const long units = static_cast<long>(a.T) * ((a.n_heads + HPS - 1) / HPS);  // < 2^31
+  const long warps_per_block = kRopeThreads / 32;
+  long grid = (units + warps_per_block - 1) / warps_per_block;
+  static int resident[64] = {0};  // blocks per SM, per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (resident[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, inv_rope_fp8_kernel<EPL, kStyle>,
+                                                      kRopeThreads, 0) != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = 1;
+    }
+    resident[dev] = n;
+  }
+  const long cap = static_cast<long>(num_sms) * resident[dev];
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  return launch_k(inv_rope_fp8_kernel<EPL, kStyle>, dim3(static_cast<unsigned>(grid)),
+                  dim3(kRopeThreads), 0, s, a);
+}
+
+}  // namespace
+
+cudaError_t launch_inv_rope_fp8(const RopeArgs& a, int num_sms, cudaStream_t s) {
+  const int epl = a.head_dim / 32;
+  if (a.style == 0) {
+    if (epl == 2) return launch_rope<2, 0>(a, num_sms, s);
+    if (epl == 4) return launch_rope<4, 0>(a, num_sms, s);
+    return launch_rope<8, 0>(a, num_sms, s);
+  }
+  if (epl == 2) return launch_rope<2, 1>(a, num_sms, s);
+  if (epl == 4) return launch_rope<4, 1>(a, num_sms, s);
+  return launch_rope<8, 1>(a, num_sms, s);
+}
+
+}  // namespace fmoe

@@ -18,12 +18,12 @@ capi = pytest.importorskip("mixture_experts_layer_26_b200.capi",
 
 def header_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"FMOE_API\s+[\w\s\*]+?\b(fused_moe\w*)\s*\(", text)))
+    return sorted(set(re.findall(r"FMOE_API\s+[\w\s\*]+?\b(fused_\w*)\s*\(", text)))
 
 
 def test_header_symbols_are_exported():
     syms = header_symbols()
-    assert len(syms) == 16
+    assert len(syms) == 17
     assert set(syms) == set(capi.EXPORTED)
     lib = ctypes.CDLL(capi.LIB_PATH)
     for s in syms:
@@ -203,3 +203,30 @@ def test_routing_descriptor_validation():
     assert call_fused(capi.make_dims(4, 256, 512, 8, 2, True, routing=bad)) == capi.FMOE_ERR_INVALID_ARG
     softmax = capi.FmoeRouting(capi.FMOE_ROUTE_SOFTMAX, 0, 0, 0.0, None)
     assert call_fused(capi.make_dims(4, 256, 512, 8, 2, True, routing=softmax)) == capi.FMOE_ERR_WORKSPACE
+
+
+def test_inv_rope_validation_makes_no_cuda_call():
+    # every rejection happens before any launch (fake pointers are never dereferenced)
+    def call(**kw):
+        args = dict(T=8, n_heads=4, head_dim=128, rot_dim=128, style=0, max_pos=64)
+        args.update(kw)
+        d = capi.make_rope_dims(**args)
+        return capi.fused_inv_rope_fp8_quant_per_head(d, _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE),
+                                                      _T(FAKE), None, stream=0, check=False)
+    inv = capi.FMOE_ERR_INVALID_ARG
+    assert call(head_dim=96) == inv                  # 64, 128 or 256 only
+    assert call(rot_dim=4) == inv                    # at least 2 * head_dim / 32
+    assert call(rot_dim=256) == inv                  # at most head_dim
+    assert call(rot_dim=96) == inv                   # style 0: a power of two
+    assert call(style=1, rot_dim=100) == inv         # style 1: a multiple of 2 * head_dim / 32
+    assert call(style=2) == inv
+    assert call(n_heads=0) == inv
+    assert call(max_pos=0) == inv
+    assert call(T=-1) == inv
+    assert call(T=0) == capi.FMOE_OK                 # nothing to do, nothing launched
+    d = capi.make_rope_dims(8, 4, 128, 128)
+    assert capi.fused_inv_rope_fp8_quant_per_head(d, None, _T(FAKE), _T(FAKE), _T(FAKE), _T(FAKE),
+                                                  None, stream=0, check=False) == inv
+    assert capi.fused_inv_rope_fp8_quant_per_head(d, _T(FAKE + 8), _T(FAKE), _T(FAKE), _T(FAKE),
+                                                  _T(FAKE), None, stream=0,
+                                                  check=False) == capi.FMOE_ERR_UNSUPPORTED
