@@ -363,6 +363,42 @@ def run_ours(args, rank, world, local_rank):
     ms_step = ms / args.steps
     value = tokens_per_second(world, s.T, args.steps, ms)
 
+    # ---- per-call distribution (events around every call) and a CUDA-graph replay of the
+    # same call; both after the timed region, neither feeds `value`
+    n_calls = max(5, min(args.steps, 200))
+    call_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_calls)]
+    for c0, c1 in call_ev:
+        c0.record(stream)
+        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+        c1.record(stream)
+    torch.cuda.synchronize()
+    per_call = sorted(c0.elapsed_time(c1) for c0, c1 in call_ev)
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, side)  # warm-up on the side stream
+        stream.wait_stream(side)
+        with torch.cuda.graph(g, stream=side):
+            capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, side)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(n_calls):
+            g.replay()
+        r1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = r0.elapsed_time(r1) / n_calls
+        del g
+    except RuntimeError as exc:  # capture unsupported in this environment: report, go on
+        print(f"graph replay skipped: {exc}", file=sys.stderr)
+    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+
     # ---- per-kernel times (events after every launch), same inputs, after the timed region
     nprof = max(5, min(args.steps, 200))
     per = {}
@@ -471,6 +507,10 @@ def run_ours(args, rank, world, local_rank):
                 "api": "fused_moe_host_io (pinned host x and out)"},
         "gpu_launches": capi.fused_moe_launches_per_call(dims) * args.steps,
         "clocks": clocks,
+        "per_call_ms": {"calls": n_calls, "median": round(statistics.median(per_call), 5),
+                        "p95": round(per_call[min(n_calls - 1, int(0.95 * n_calls))], 5),
+                        "note": "events around each call, after the timed region"},
+        "graph_replay_ms_per_call": None if graph_ms is None else round(graph_ms, 5),
     }
     print(json.dumps(line))
     return 0

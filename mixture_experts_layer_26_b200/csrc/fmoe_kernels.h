@@ -20,7 +20,10 @@ inline cudaError_t set_max_dynamic_smem(int bytes) {
   const unsigned bit = 1u << (dev & 31);
   if (configured & bit) return cudaSuccess;
   err = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (err == cudaSuccess) configured |= bit;
+  if (err == cudaSuccess)
+    configured |= bit;
+  else
+    (void)cudaGetLastError();  // reported here; must not surface at a later launch check
   return err;
 }
 

@@ -48,125 +48,20 @@ __device__ __forceinline__ float sigmoid_f64(float l) {
   return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(l))));
 }
 
-template <int TB, int EG>
-__global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                    // [TB][H]
-  float* logits = reinterpret_cast<float*>(smem + TB * a.H * 2);       // [TB][E]
-  __shared__ float red[kRouterThreads / 32];
+// After the logits: the hand-off of a split token tile to its last CTA, top-k and the
+// routing weights (one warp per token), and -- one-call path, small batches -- the
+// permutation, plan and gather by the CTA that finishes the last token tile.  `logits`
+// is [TB][E] (and [TB][E] of grouped selection scores after it) in shared memory; when
+// the experts are split over CTAs the tile's logits are in a.logits_g.  The dynamic
+// shared memory from `smem` on is reused by the permutation.
+template <int TB>
+__device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, int tile,
+                            bool split) {
   __shared__ int is_last;
   __shared__ int is_final;
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, group = blockIdx.y;
   const int t0 = tile * TB;
-  const int H = a.H, E = a.E;
-  const int vec_per_row = H / 8;  // 16-byte vectors per row
-  const bool split = gridDim.y > 1;
-
-  griddep_wait();
-  griddep_launch_dependents();
-
-  // ---- stage x rows (zero for tokens past T) and their max |x|
-  float amax = 0.f;
-  for (int i = threadIdx.x; i < TB * vec_per_row; i += kRouterThreads) {
-    const int t = i / vec_per_row, v = i % vec_per_row;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (t0 + t < a.T)
-      val = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + t) * H) + v);
-    reinterpret_cast<uint4*>(xs + t * H)[v] = val;
-    const uint32_t w4[4] = {val.x, val.y, val.z, val.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(w4[j] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(w4[j] & 0xFFFF0000u)));
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  if (lane == 0) red[warp] = amax;
-  __syncthreads();
-  if (threadIdx.x == 0 && group == 0) {
-    float m = 0.f;
-    for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, red[w]);
-    a.amax_part[tile] = m;
-    if (tile == 0) a.hdr->router_ctas = gridDim.x;
-  }
-
-  // ---- logits of this CTA's experts, in the canonical order
-  const int steps = H / 256;  // chunks per lane
-  const int e_begin = group * a.experts_per_cta;
-  const int e_end = min(E, e_begin + a.experts_per_cta);
-  // chunk steps whose router rows are loaded together: more when a warp owns fewer
-  // experts, so that every warp keeps about eight 16-byte loads in flight
-  constexpr int U = EG >= 4 ? 2 : 8 / EG;
-  // Accumulators acc[t][g] are updated in pairs with one paired FMA (each component
-  // rounds exactly like a scalar fmaf), element by element in ascending order, so
-  // every logit keeps the canonical summation order.
-  constexpr int NACC = TB * EG;
-  constexpr bool kPairG = (EG % 2 == 0);  // pairs (t, g), (t, g+1); else (t, g), (t+1, g)
-  for (int eb = e_begin + warp * EG; eb < e_end; eb += (kRouterThreads / 32) * EG) {
-    float acc[TB][EG];
-#pragma unroll
-    for (int t = 0; t < TB; ++t)
-#pragma unroll
-      for (int g = 0; g < EG; ++g) acc[t][g] = 0.f;
-    for (int s0 = 0; s0 < steps; s0 += U) {
-      uint4 wv[U][EG];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int g = 0; g < EG; ++g) {
-          const int e = min(eb + g, e_end - 1);
-          const int chunk = lane + 32 * min(s0 + u, steps - 1);
-          wv[u][g] = __ldg(reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H) + chunk);
-        }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (s0 + u < steps) {
-          const int chunk = lane + 32 * (s0 + u);
-          float wf[EG][8], xf[TB][8];
-#pragma unroll
-          for (int g = 0; g < EG; ++g) unpack8(wv[u][g], wf[g]);
-#pragma unroll
-          for (int t = 0; t < TB; ++t) unpack8(reinterpret_cast<const uint4*>(xs + t * H)[chunk], xf[t]);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if constexpr (NACC % 2 == 0) {
-#pragma unroll
-              for (int m = 0; m < NACC; m += 2) {
-                const int ta = m / EG, ga = m % EG;
-                const int tb = kPairG ? ta : ta + 1, gb = kPairG ? ga + 1 : ga;
-                const float2 r = __ffma2_rn(make_float2(xf[ta][i], xf[tb][i]),
-                                            make_float2(wf[ga][i], wf[gb][i]),
-                                            make_float2(acc[ta][ga], acc[tb][gb]));
-                acc[ta][ga] = r.x;
-                acc[tb][gb] = r.y;
-              }
-            } else {
-              acc[0][0] = __fmaf_rn(xf[0][i], wf[0][i], acc[0][0]);
-            }
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < TB; ++t)
-#pragma unroll
-      for (int g = 0; g < EG; ++g) {
-        float p = acc[t][g];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) p = p + __shfl_xor_sync(0xffffffffu, p, off);
-        if (lane == 0 && eb + g < e_end) {
-          if (split) {
-            if (t0 + t < a.T) a.logits_g[static_cast<size_t>(t0 + t) * E + eb + g] = p;
-          } else {
-            logits[t * E + eb + g] = p;
-          }
-        }
-      }
-  }
-
+  const int E = a.E;
   if (split) {
     // The last of the gridDim.y CTAs of this token tile to finish picks the top-k
     // (counter reset for the next call by that CTA).
@@ -319,6 +214,126 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
       gather_rows(a.gather, warp, kRouterThreads / 32);
     }
   }
+}
+
+template <int TB, int EG>
+__global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                    // [TB][H]
+  float* logits = reinterpret_cast<float*>(smem + TB * a.H * 2);       // [TB][E]
+  __shared__ float red[kRouterThreads / 32];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, group = blockIdx.y;
+  const int t0 = tile * TB;
+  const int H = a.H, E = a.E;
+  const int vec_per_row = H / 8;  // 16-byte vectors per row
+  const bool split = gridDim.y > 1;
+
+  griddep_wait();
+  griddep_launch_dependents();
+
+  // ---- stage x rows (zero for tokens past T) and their max |x|
+  float amax = 0.f;
+  for (int i = threadIdx.x; i < TB * vec_per_row; i += kRouterThreads) {
+    const int t = i / vec_per_row, v = i % vec_per_row;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (t0 + t < a.T)
+      val = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + t) * H) + v);
+    reinterpret_cast<uint4*>(xs + t * H)[v] = val;
+    const uint32_t w4[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w4[j] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w4[j] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0 && group == 0) {
+    float m = 0.f;
+    for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, red[w]);
+    a.amax_part[tile] = m;
+    if (tile == 0) a.hdr->router_ctas = gridDim.x;
+  }
+
+  // ---- logits of this CTA's experts, in the canonical order
+  const int steps = H / 256;  // chunks per lane
+  const int e_begin = group * a.experts_per_cta;
+  const int e_end = min(E, e_begin + a.experts_per_cta);
+  // chunk steps whose router rows are loaded together: more when a warp owns fewer
+  // experts, so that every warp keeps about eight 16-byte loads in flight
+  constexpr int U = EG >= 4 ? 2 : 8 / EG;
+  // Accumulators acc[t][g] are updated in pairs with one paired FMA (each component
+  // rounds exactly like a scalar fmaf), element by element in ascending order, so
+  // every logit keeps the canonical summation order.
+  constexpr int NACC = TB * EG;
+  constexpr bool kPairG = (EG % 2 == 0);  // pairs (t, g), (t, g+1); else (t, g), (t+1, g)
+  for (int eb = e_begin + warp * EG; eb < e_end; eb += (kRouterThreads / 32) * EG) {
+    float acc[TB][EG];
+#pragma unroll
+    for (int t = 0; t < TB; ++t)
+#pragma unroll
+      for (int g = 0; g < EG; ++g) acc[t][g] = 0.f;
+    for (int s0 = 0; s0 < steps; s0 += U) {
+      uint4 wv[U][EG];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int g = 0; g < EG; ++g) {
+          const int e = min(eb + g, e_end - 1);
+          const int chunk = lane + 32 * min(s0 + u, steps - 1);
+          wv[u][g] = __ldg(reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H) + chunk);
+        }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (s0 + u < steps) {
+          const int chunk = lane + 32 * (s0 + u);
+          float wf[EG][8], xf[TB][8];
+#pragma unroll
+          for (int g = 0; g < EG; ++g) unpack8(wv[u][g], wf[g]);
+#pragma unroll
+          for (int t = 0; t < TB; ++t) unpack8(reinterpret_cast<const uint4*>(xs + t * H)[chunk], xf[t]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if constexpr (NACC % 2 == 0) {
+#pragma unroll
+              for (int m = 0; m < NACC; m += 2) {
+                const int ta = m / EG, ga = m % EG;
+                const int tb = kPairG ? ta : ta + 1, gb = kPairG ? ga + 1 : ga;
+                const float2 r = __ffma2_rn(make_float2(xf[ta][i], xf[tb][i]),
+                                            make_float2(wf[ga][i], wf[gb][i]),
+                                            make_float2(acc[ta][ga], acc[tb][gb]));
+                acc[ta][ga] = r.x;
+                acc[tb][gb] = r.y;
+              }
+            } else {
+              acc[0][0] = __fmaf_rn(xf[0][i], wf[0][i], acc[0][0]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TB; ++t)
+#pragma unroll
+      for (int g = 0; g < EG; ++g) {
+        float p = acc[t][g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) p = p + __shfl_xor_sync(0xffffffffu, p, off);
+        if (lane == 0 && eb + g < e_end) {
+          if (split) {
+            if (t0 + t < a.T) a.logits_g[static_cast<size_t>(t0 + t) * E + eb + g] = p;
+          } else {
+            logits[t * E + eb + g] = p;
+          }
+        }
+      }
+  }
+
+  router_tail<TB>(a, smem, logits, tile, split);
 }
 
 template <int TB, int EG>

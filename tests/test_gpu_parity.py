@@ -142,6 +142,12 @@ SMALL = [
     ("fp8_grouped_shared", (64, 512, 256, 64, 8, "fp8"),
      {"router_std": 1.0, "grouped": (8, 4, 2.5), "n_shared": 1}),
     ("fp8_shared_pair_chunks", (300, 256, 256, 4, 2, "fp8"), {"n_shared": 1}),
+    # E >= 128: four experts per router warp, experts split over CTAs (last-CTA hand-off),
+    # a last expert group that is not full, grouped routing with a shared expert
+    ("fp8_experts_128", (13, 512, 256, 128, 4, "fp8"), {"router_std": 1.0}),
+    ("fp8_experts_130", (9, 1024, 128, 130, 3, "fp8"), {}),
+    ("bf16_grouped_shared_160", (20, 1024, 256, 160, 6, "bf16"),
+     {"grouped": (8, 3, 1.5), "n_shared": 1}),
 ]
 
 
