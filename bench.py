@@ -214,8 +214,14 @@ def oracle_full_pass(inp):
 
 
 class OracleSlices:
-    """Bounded steps of the oracle: the expert networks of one touched expert over the
-    whole token batch per step, plus routing / permutation / combine once per cycle."""
+    """Bounded steps of the oracle.  A step runs the oracle's expert networks for one
+    touched expert over all of its rows, restricted to a block of F intermediate features
+    (the gate/up rows and the w2 columns of those features: the same computation on a
+    narrower expert); F is chosen so that a step costs a few tens of milliseconds.  The
+    layer is all (expert, feature block) slices plus routing, permutation and combine,
+    which are timed once."""
+
+    WORK_PER_STEP = 384e6  # weight elements decoded + row x weight products, per step
 
     def __init__(self, inp):
         from oracle import fused_moe_oracle as O
@@ -235,18 +241,30 @@ class OracleSlices:
         self.prep = (ids, w, counts, offsets, rows, inv, a_perm, s1)
         self.fixed_s = time.perf_counter() - t0
         self.touched = [e for e in range(s.E_all) if counts[e] > 0]
+        # feature blocks: (expert, f0, f1), F a multiple of 64 dividing into I
+        self.slices = []
+        for e in self.touched:
+            n = int(counts[e])
+            F = int(self.WORK_PER_STEP / (3.0 * s.H * (n + 64)))
+            F = max(64, min(s.I, F // 64 * 64))
+            self.slices += [(e, f0, min(s.I, f0 + F)) for f0 in range(0, s.I, F)]
         self.i = 0
 
     def step(self):
         s, d, O = self.inp.shape, self.d, self.O
         ids, w, counts, offsets, rows, inv, a_perm, s1 = self.prep
-        e = self.touched[self.i % len(self.touched)]
+        e, f0, f1 = self.slices[self.i % len(self.slices)]
         self.i += 1
-        offs = np.zeros_like(offsets)
-        offs[e + 1:] = offsets[e + 1] - offsets[e]
         r0, r1 = offsets[e], offsets[e + 1]
-        O.experts(a_perm[r0:r1], offs, rows[r0:r1], w, d["w13"], d["w2"], s.H, s.I, s.E_all,
-                  d["fp8"], s1, d["w13_scale"], d["w2_scale"])
+        offs = np.zeros(2, dtype=offsets.dtype)
+        offs[1] = r1 - r0
+        w13 = d["w13"][e:e + 1]
+        w13 = np.concatenate([w13[:, f0:f1], w13[:, s.I + f0:s.I + f1]], axis=1)
+        w2 = d["w2"][e:e + 1, :, f0:f1]
+        sc13 = None if d["w13_scale"] is None else d["w13_scale"][e:e + 1]
+        sc2 = None if d["w2_scale"] is None else d["w2_scale"][e:e + 1]
+        return e, O.experts(a_perm[r0:r1], offs, rows[r0:r1], w, w13, w2, s.H, f1 - f0, 1,
+                            d["fp8"], s1, sc13, sc2)[0]
 
     def combine_seconds(self):
         s = self.inp.shape
@@ -270,7 +288,7 @@ def run_reference(args, rank):
     for _ in range(args.steps):
         sl.step()
     dt = time.perf_counter() - t0
-    cycles = args.steps / len(sl.touched)
+    cycles = args.steps / len(sl.slices)  # layers' worth of expert work timed
     total = dt + cycles * (sl.fixed_s + sl.combine_seconds())
     value = s.T * cycles / total
     line = {
@@ -281,9 +299,11 @@ def run_reference(args, rank):
         "data": "synthetic", "config": workload_config(s, "oracle"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle",
-                         "sample": f"{args.steps} steps, each the expert networks of one of the "
-                                   f"{len(sl.touched)} touched experts over all T={s.T} tokens; "
-                                   "routing/permutation/combine added once per expert cycle; "
+                         "sample": f"{args.steps} steps, each the expert networks of one "
+                                   f"(touched expert, block of intermediate features) slice, "
+                                   f"{len(sl.slices)} slices per layer over "
+                                   f"{len(sl.touched)} touched experts and all T={s.T} tokens; "
+                                   "routing/permutation/combine added once per layer; "
                                    f"{warm} of the {args.warmup} warm-up steps executed"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
