@@ -42,7 +42,7 @@ bit for bit:
   * quantisation multiplies by the fp32 inverse scale in fp32 and rounds the
     fp32 product to e4m3 (round to nearest even, saturating to +-448).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   R1 canonical fp32 summation order of the router logits (see router_logits)
   R2 top-k ties go to the lower expert index; selection is on logits
   R3 permutation is stable by (expert, flattened index t*k+j)

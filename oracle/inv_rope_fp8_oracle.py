@@ -23,7 +23,7 @@ change) but give no formula, layout or shape.  The plainest reading of the name:
      q = e4m3(y * 448/amax) rounded to nearest even, saturating; amax == 0 gives
      scale 1.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   P1 the rotary table is an input: cos_sin [max_pos, rot_dim] fp32 holding the rot_dim/2
      cosines then the rot_dim/2 sines of each position (the cache layout rotary
      embeddings keep); positions [T] int32 index it;
