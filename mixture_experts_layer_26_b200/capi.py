@@ -158,12 +158,20 @@ def make_dims(T: int, H: int, I: int, E: int, top_k: int, fp8: bool, variant: st
     return d
 
 
-def dims_of(x: torch.Tensor, w13: torch.Tensor, top_k: int, variant: str = "auto") -> FmoeDims:
-    """Dims from x [T,H] and w13 [E,2I,H] (uint8 = e4m3 bytes, bfloat16 = bf16)."""
+def dims_of(x: torch.Tensor, router_w: torch.Tensor, w13: torch.Tensor, top_k: int,
+            variant: str = "auto", routing: Optional[FmoeRouting] = None) -> FmoeDims:
+    """Dims from x [T,H], router_w [E,H] and w13 [E+S,2I,H] (uint8 = e4m3 bytes, bfloat16 =
+    bf16), where S = routing.n_shared shared experts follow the E routed ones."""
     T, H = x.shape
-    E, twoI, H2 = w13.shape
-    assert H2 == H and twoI % 2 == 0
-    return make_dims(T, H, twoI // 2, E, top_k, w13.dtype == torch.uint8, variant)
+    E, H1 = router_w.shape
+    EA, twoI, H2 = w13.shape
+    n_shared = routing.n_shared if routing is not None else 0
+    if H1 != H or H2 != H or twoI % 2 != 0:
+        raise ValueError(f"shapes do not match: x {tuple(x.shape)}, router_w "
+                         f"{tuple(router_w.shape)}, w13 {tuple(w13.shape)}")
+    if EA != E + n_shared:
+        raise ValueError(f"w13 holds {EA} experts, expected E + n_shared = {E + n_shared}")
+    return make_dims(T, H, twoI // 2, E, top_k, w13.dtype == torch.uint8, variant, routing)
 
 
 def make_scales(w13_scale=None, w2_scale=None, a1_scale: float = 0.0, a2_scale: float = 0.0) -> FmoeScales:
@@ -332,3 +340,19 @@ def fused_inv_rope_fp8_quant_per_head(dims: FmoeRopeDims, x, positions, cos_sin,
     st = _inv_rope(ctypes.byref(dims), _ptr(x), _ptr(positions), _ptr(cos_sin), _ptr(q),
                    _ptr(scales), _ptr(device_status), _stream(stream))
     return _check(st, "fused_inv_rope_fp8_quant_per_head") if check else st
+
+
+def moe(x: torch.Tensor, router_w: torch.Tensor, w13: torch.Tensor, w2: torch.Tensor, top_k: int,
+        w13_scale=None, w2_scale=None, out: Optional[torch.Tensor] = None,
+        routing: Optional[FmoeRouting] = None, a1_scale: float = 0.0, a2_scale: float = 0.0,
+        variant: str = "auto", ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The whole layer on device tensors in one call: dims from the shapes, a workspace
+    allocated when none is given, out [T,H] bf16 allocated when none is given."""
+    dims = dims_of(x, router_w, w13, top_k, variant, routing)
+    if ws is None:
+        ws = alloc_workspace(dims, x.device)
+    if out is None:
+        out = torch.empty(x.shape[0], x.shape[1], dtype=torch.bfloat16, device=x.device)
+    fused_moe(dims, x, router_w, w13, w2, make_scales(w13_scale, w2_scale, a1_scale, a2_scale),
+              out, ws, stream)
+    return out

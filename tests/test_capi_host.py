@@ -230,3 +230,17 @@ def test_inv_rope_validation_makes_no_cuda_call():
     assert capi.fused_inv_rope_fp8_quant_per_head(d, _T(FAKE + 8), _T(FAKE), _T(FAKE), _T(FAKE),
                                                   _T(FAKE), None, stream=0,
                                                   check=False) == capi.FMOE_ERR_UNSUPPORTED
+
+
+def test_dims_from_tensor_shapes():
+    import torch
+    x = torch.empty(5, 256, dtype=torch.bfloat16)
+    wr = torch.empty(8, 256, dtype=torch.bfloat16)
+    w13 = torch.empty(9, 1024, 256, dtype=torch.uint8)      # 8 routed + 1 shared, I = 512
+    r = capi.make_softmax_routing(1)
+    d = capi.dims_of(x, wr, w13, 2, routing=r)
+    assert (d.T, d.H, d.I, d.E, d.top_k, d.wdtype) == (5, 256, 512, 8, 2, capi.FMOE_FP8_E4M3)
+    with pytest.raises(ValueError):
+        capi.dims_of(x, wr, w13, 2)                          # a shared expert without routing
+    with pytest.raises(ValueError):
+        capi.dims_of(x, torch.empty(8, 128, dtype=torch.bfloat16), w13, 2, routing=r)

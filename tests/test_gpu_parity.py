@@ -208,6 +208,18 @@ def test_pair_variant_equals_normal(small_cases, name):
     assert np.array_equal(out_n, out_p)
 
 
+@pytest.mark.parametrize("name", ["fp8_ragged", "fp8_shared", "bf16_grouped_shared_160"])
+def test_tensor_level_call_equals_dims_call(small_cases, name):
+    """capi.moe (dims from the tensor shapes, its own workspace) gives the same bits as
+    fused_moe with explicit dims."""
+    inp, g, ref = small_cases(name)
+    out_d, _ = run_fused(inp, g, "auto")
+    out_t = capi.moe(g["x"], g["router_w"], g["w13"], g["w2"], inp.shape.top_k,
+                     g["w13_scale"], g["w2_scale"], routing=g.get("routing"))
+    torch.cuda.synchronize()
+    assert np.array_equal(bits16(out_t), out_d)
+
+
 def test_static_scales(small_cases):
     inp, g, _ = small_cases("fp8_ragged")
     ref = run_oracle(O, inp, a1_scale=0.02, a2_scale=0.003)
