@@ -32,3 +32,33 @@ def test_slices_cover_the_layer_and_add_up(monkeypatch):
         e, y = sl2.step()
         y_sum[offsets[e]:offsets[e + 1]] += y
     assert np.abs(y_sum - y_full).max() <= 1e-9 * np.abs(y_full).max()
+
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("workload", ["tiny_bf16", "inv_rope_fp8_partial"])
+def test_reference_arm_prints_one_contract_line(workload):
+    """`bench.py --impl reference` runs the oracle on the host cores only and prints one
+    JSON line with the contract's keys (the end-to-end number equals the value, no copies)."""
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
+                        "--steps", "2", "--warmup", "3"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "cpu_baseline", "e2e", "config"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 2
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"]["value"] == j["value"]
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
