@@ -348,6 +348,13 @@ def moe(x: torch.Tensor, router_w: torch.Tensor, w13: torch.Tensor, w2: torch.Te
         variant: str = "auto", ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """The whole layer on device tensors in one call: dims from the shapes, a workspace
     allocated when none is given, out [T,H] bf16 allocated when none is given."""
+    for name, t in (("x", x), ("router_w", router_w), ("w13", w13), ("w2", w2)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if x.dtype != torch.bfloat16 or router_w.dtype != torch.bfloat16:
+        raise ValueError("x and router_w must be bfloat16")
+    if w2.dtype != w13.dtype or w13.dtype not in (torch.uint8, torch.bfloat16):
+        raise ValueError("w13 and w2 must both be uint8 (e4m3 bytes) or both bfloat16")
     dims = dims_of(x, router_w, w13, top_k, variant, routing)
     if ws is None:
         ws = alloc_workspace(dims, x.device)

@@ -244,3 +244,13 @@ def test_dims_from_tensor_shapes():
         capi.dims_of(x, wr, w13, 2)                          # a shared expert without routing
     with pytest.raises(ValueError):
         capi.dims_of(x, torch.empty(8, 128, dtype=torch.bfloat16), w13, 2, routing=r)
+
+
+def test_tensor_level_call_rejects_bad_tensors_before_any_cuda_call():
+    import torch
+    x = torch.empty(5, 256, dtype=torch.bfloat16)      # CPU tensors: rejected up front
+    wr = torch.empty(8, 256, dtype=torch.bfloat16)
+    w13 = torch.empty(8, 1024, 256, dtype=torch.uint8)
+    w2 = torch.empty(8, 256, 512, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        capi.moe(x, wr, w13, w2, 2)
