@@ -96,58 +96,74 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
 
   // Software pipeline over this warp's units u, u + nwarps, ...: the position of unit
   // u + 2*nwarps and the x rows and table entries of unit u + nwarps are in flight while
-  // unit u is rotated, quantised and stored.
+  // unit u is rotated, quantised and stored.  Unit u is (token u / hgroups, head group
+  // u % hgroups); the three units in flight carry their indices forward by nwarps.
   struct Unit {
-    int t, h0;
+    int t, hg;
   };
-  auto unit_of = [&](int u) { return Unit{u / hgroups, (u % hgroups) * HPS}; };
-  auto pos_of = [&](int u) -> int {
-    if (u >= units) return 0;
-    const Unit w = unit_of(u);
+  const int dq = nwarps / hgroups, dr = nwarps % hgroups;
+  auto advance = [&](Unit w) {
+    w.t += dq;
+    w.hg += dr;
+    if (w.hg >= hgroups) {
+      w.hg -= hgroups;
+      ++w.t;
+    }
+    return w;
+  };
+  auto pos_of = [&](Unit w) -> int {
+    if (w.t >= a.T) return 0;
     int p = __ldg(a.positions + w.t);
     if (p < 0 || p >= a.max_pos) {
-      if (lane == 0 && w.h0 == 0 && a.status != nullptr) record_status(a.status, ST_BOUNDS);
+      if (lane == 0 && w.hg == 0 && a.status != nullptr) record_status(a.status, ST_BOUNDS);
       p = 0;
     }
     return p;
   };
-  auto load_x = [&](int u, XV (&xv)[HPS]) {
-    if (u >= units) return;
-    const Unit w = unit_of(u);
+  auto load_x = [&](Unit w, XV (&xv)[HPS]) {
+    if (w.t >= a.T) return;
+    const int h0 = w.hg * HPS;
     const XV* src = reinterpret_cast<const XV*>(
-        a.x + (static_cast<size_t>(w.t) * a.n_heads + w.h0) * hd + j0);
+        a.x + (static_cast<size_t>(w.t) * a.n_heads + h0) * hd + j0);
 #pragma unroll
     for (int k = 0; k < HPS; ++k)
-      if (w.h0 + k < a.n_heads) xv[k] = __ldcs(src + k * 32);  // streamed once
+      if (h0 + k < a.n_heads) xv[k] = __ldcs(src + k * 32);  // streamed once
   };
-  auto load_table = [&](int u, int p, float (&cs)[NC], float (&sn)[NC]) {
-    if (u >= units || !rotated) return;
+  // the sines come pre-negated for the b coordinates of a half-split pair, so that every
+  // rotated coordinate is fadd(fmul(x, cos), fmul(partner, sin')): for b that is
+  // -(x_a*sin) + x_b*cos exactly (IEEE addition commutes and negation is exact)
+  auto load_table = [&](Unit w, int p, float (&cs)[NC], float (&sn)[NC]) {
+    if (w.t >= a.T || !rotated) return;
     const float* row = a.cos_sin + static_cast<size_t>(p) * rot;
     load_row<NC>(row + i0, cs);
     load_row<NC>(row + half + i0, sn);
+    if (kStyle == 0 && !is_a) {
+#pragma unroll
+      for (int i = 0; i < NC; ++i) sn[i] = -sn[i];
+    }
   };
 
-  int u = gwarp;
+  if (gwarp >= units) return;
+  Unit uc{gwarp / hgroups, gwarp % hgroups};
+  Unit un = advance(uc), ua = advance(un);
   XV xc[HPS], xn[HPS];
   float cc[NC], sc_[NC], cn[NC], sn_[NC];
-  int p_next = pos_of(u + nwarps);
-  {
-    const int p0 = pos_of(u);
-    load_x(u, xc);
-    load_table(u, p0, cc, sc_);
-  }
-  for (; u < units; u += nwarps) {
+  for (int i = 0; i < NC; ++i) cc[i] = sc_[i] = cn[i] = sn_[i] = 0.f;
+  int p_next = pos_of(un);
+  load_x(uc, xc);
+  load_table(uc, pos_of(uc), cc, sc_);
+  while (uc.t < a.T) {
     // next unit's x and table (its position is already here), the one after's position
-    load_x(u + nwarps, xn);
-    load_table(u + nwarps, p_next, cn, sn_);
-    const int p_after = pos_of(u + 2 * nwarps);
+    load_x(un, xn);
+    load_table(un, p_next, cn, sn_);
+    const int p_after = pos_of(ua);
 
-    const Unit w = unit_of(u);
-    uint8_t* qdst = a.q + (static_cast<size_t>(w.t) * a.n_heads + w.h0) * hd + j0;
-    float* sdst = a.scales + static_cast<size_t>(w.t) * a.n_heads + w.h0;
+    const int h0 = uc.hg * HPS;
+    uint8_t* qdst = a.q + (static_cast<size_t>(uc.t) * a.n_heads + h0) * hd + j0;
+    float* sdst = a.scales + static_cast<size_t>(uc.t) * a.n_heads + h0;
 #pragma unroll
     for (int k = 0; k < HPS; ++k) {
-      if (w.h0 + k >= a.n_heads) break;  // warp-uniform
+      if (h0 + k >= a.n_heads) break;  // warp-uniform
       float x[EPL], y[EPL];
       unpack_bf16<EPL>(xc[k], x);
       if constexpr (kStyle == 0) {
@@ -162,25 +178,17 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
         }
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
-          if (!rotated) {
-            y[e] = x[e];
-          } else if (is_a) {  // x[e] = x_a, o = x_b
-            y[e] = __fadd_rn(__fmul_rn(x[e], cc[e]), __fmul_rn(o[e], sc_[e]));
-          } else {            // x[e] = x_b, o = x_a
-            y[e] = __fadd_rn(-__fmul_rn(o[e], sc_[e]), __fmul_rn(x[e], cc[e]));
-          }
+          const float r = __fadd_rn(__fmul_rn(x[e], cc[e]), __fmul_rn(o[e], sc_[e]));
+          y[e] = rotated ? r : x[e];
         }
       } else {
 #pragma unroll
         for (int e = 0; e < EPL; e += 2) {
-          if (!rotated) {
-            y[e] = x[e];
-            y[e + 1] = x[e + 1];
-          } else {
-            const float c = cc[e / 2], s = sc_[e / 2];
-            y[e] = __fadd_rn(__fmul_rn(x[e], c), __fmul_rn(x[e + 1], s));
-            y[e + 1] = __fadd_rn(-__fmul_rn(x[e], s), __fmul_rn(x[e + 1], c));
-          }
+          const float c = cc[e / 2], sn = sc_[e / 2];
+          const float r0 = __fadd_rn(__fmul_rn(x[e], c), __fmul_rn(x[e + 1], sn));
+          const float r1 = __fadd_rn(__fmul_rn(x[e + 1], c), __fmul_rn(x[e], -sn));
+          y[e] = rotated ? r0 : x[e];
+          y[e + 1] = rotated ? r1 : x[e + 1];
         }
       }
       // max |y| over the head: the bit patterns of non-negative finite floats order like
@@ -207,6 +215,9 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
       sc_[i] = sn_[i];
     }
     p_next = p_after;
+    uc = un;
+    un = ua;
+    ua = advance(ua);
   }
 }
 
