@@ -254,3 +254,37 @@ def test_tensor_level_call_rejects_bad_tensors_before_any_cuda_call():
     w2 = torch.empty(8, 256, 512, dtype=torch.uint8)
     with pytest.raises(ValueError):
         capi.moe(x, wr, w13, w2, 2)
+
+
+def test_host_properties_over_many_dims():
+    """Host-only properties over a grid of dims: the workspace holds at least the routed
+    rows' buffers, the launch count follows the documented rule, invalid dims report
+    size 0.  (The size is not monotone in T: the swap-AB variant also holds split-K
+    partials, capped at 64 MB per contraction, which the normal variants do not.)"""
+    import itertools
+    rules = 0
+    for (H, I), (E, k), fp8, variant, ns in itertools.product(
+            [(256, 128), (4096, 1024), (7168, 2048)], [(8, 2), (64, 6), (256, 8)],
+            [True, False], ["auto", "swap_ab", "normal", "normal_pair"], [0, 1]):
+        r = capi.make_softmax_routing(ns) if ns else None
+        for T in (1, 7, 64, 300, 2048):
+            d = capi.make_dims(T, H, I, E, k, fp8, variant, routing=r)
+            R = T * (k + ns)
+            # at least the permuted activations, y and hq of every routed row
+            es = 1 if fp8 else 2
+            assert capi.workspace_size(d) >= R * H * (es + 4) + R * I * es
+            # variant the library resolves for AUTO: <= 64 rows per expert on average ->
+            # swap-AB, else the normal tiles (one CTA or pairs)
+            swap = variant == "swap_ab" or (variant == "auto" and (R + E + ns - 1) // (E + ns) <= 64)
+            n = 4 + (1 if fp8 else 0) + (1 if swap else 0)
+            if R > 2048:
+                n += 2
+            elif R * H * 2 > 128 * 1024:
+                n += 1
+            assert capi.fused_moe_launches_per_call(d) == n, (T, H, I, E, k, fp8, variant, ns)
+            rules += 1
+    assert rules == 3 * 3 * 2 * 4 * 2 * 5
+    for bad in (dict(E=257), dict(k=0), dict(H=300), dict(I=100)):
+        kw = dict(T=4, H=256, I=128, E=8, k=2)
+        kw.update(bad)
+        assert capi.workspace_size(capi.make_dims(kw["T"], kw["H"], kw["I"], kw["E"], kw["k"], True)) == 0
