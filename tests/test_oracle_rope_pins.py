@@ -149,3 +149,18 @@ def test_inverse_scale_is_one_division_448_over_amax():
     q, sc = RO.quant_per_head(y)
     want = torch.tensor([float(f(v * inv_a))]).to(torch.float8_e4m3fn).view(torch.uint8).item()
     assert q[0, 0, 1] == want and sc[0, 0] == f(a / f(448))
+
+
+def test_tiny_regression_golden():
+    """The oracle against its own committed record (tests/golden/make_golden_rope.py):
+    catches an unintended change of the oracle's arithmetic, not a wrong reading."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "inv_rope_tiny_seed0.json")
+    doc = json.load(open(path))
+    s = minp.RopeShape(**doc["shape"])
+    inp = minp.make_rope_inputs(s, seed=0)
+    r = RO.inv_rope_fp8_quant(minp.bf16_bits(inp.x), inp.positions.numpy(), inp.cos_sin.numpy(),
+                              s.rot_dim, s.style)
+    assert r["q"].tolist() == doc["codes"]
+    assert [[float(v) for v in row] for row in r["scales"]] == doc["scales"]
