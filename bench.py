@@ -2,29 +2,33 @@
 """Benchmark of the fused MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload mixtral_fp8_decode] [--T 64]
+                    [--workload prefill_fp8] [--T 4096]
 
 A step is one call of the whole layer (route -> permute/quantise -> both expert
-contractions -> combine) through the C ABI on one batch of T tokens; the default
-workload is the Mixtral-like FP8 decode shape (H=4096, I=14336, E=8, top_k=2) at
-T=64.  Inputs are seeded synthetic tensors resident in HBM; the expert weights
-(1.41 GB) exceed the 126 MB L2, so no L2 flush is needed between steps.  W
-untimed warm-up steps, then exactly K steps timed with CUDA events on the
-launching stream between a barrier + synchronize on both sides; the time is the
-max over ranks.  For N > 1 every rank runs an independent replica of the layer
-(the single-GPU layer has no exchange step) and `value` is the tokens of all
-ranks divided by that time.
+contractions -> combine) through the C ABI on one batch of T tokens.  The default
+workload is the largest single-GPU configuration: the FP8 prefill batch of T=4096 tokens
+on Mixtral-like shapes (H=4096, I=14336, E=8, top_k=2), bound by the FP8 tensor pipe.
+Inputs are seeded synthetic tensors resident in HBM; the expert weights (1.41 GB)
+exceed the 126 MB L2, so no L2 flush is needed between steps.  W untimed warm-up steps,
+then exactly K steps timed with CUDA events on the launching stream between a barrier +
+synchronize on both sides; the time is the max over ranks.  For N > 1 every rank runs an
+independent replica of the layer (the single-GPU layer has no exchange step) and `value`
+is the tokens of all ranks divided by that time.
 
 Rank 0 prints one JSON line.  Besides the contract keys it reports the roofline of
 the dominant kernel (timed live per launch with CUDA events through
-fused_moe_profile), the oracle timed on the host cores (cpu_baseline), an
-end-to-end number through fused_moe_host_io with pinned host buffers, and the SM
-clocks sampled with nvidia-smi during the timed region.
+fused_moe_profile) against the burst peak of its bound (the FP8 tensor peak is measured
+in the same run with the library GEMM, torch._scaled_mm on e4m3 operands), the oracle
+timed on the host cores on a bounded sample (cpu_baseline, all cores and one core), an
+end-to-end number through fused_moe_host_io with pinned host buffers, and the SM clocks
+sampled with nvidia-smi from the timed region on.  With the default workload the line
+also carries `decode`: the HBM-bound decode regime (Mixtral-like T=64, DeepSeek-V3-like
+T=256), each measured the same way with its own roofline and end-to-end number.
 
 --impl reference times the CPU oracle (the reference arm) on the same workload:
-each step runs the oracle's expert networks for one touched expert over the full
-token batch (a bounded slice); one cycle over the touched experts plus routing and
-combine is one full layer pass.
+each step runs the oracle's expert networks for one (touched expert, block of
+intermediate features) slice over all of that expert's rows; one cycle over the slices
+plus routing and combine is one full layer pass.
 """
 from __future__ import annotations
 
@@ -49,6 +53,7 @@ import torch  # noqa: E402
 from mixture_experts_layer_26_b200 import inputs as minp  # noqa: E402
 
 METRIC = "fused-MoE tokens/s; achieved HBM GB/s (decode) / FP8 TFLOPS (prefill) vs peak"
+DEFAULT_WORKLOAD = "prefill_fp8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 2 ** 20
 # sources whose hash an ncu summary of a GEMM kernel records (pair kernels: gemm_pair.cu)
@@ -202,17 +207,6 @@ def tokens_per_second(world: int, T: int, steps: int, ms_max: float) -> float:
 
 # --------------------------------------------------------------------------- CPU oracle timing
 
-def oracle_full_pass(inp):
-    """The oracle on the whole batch once: (seconds, touched experts)."""
-    from oracle import fused_moe_oracle as O
-    d = np_inputs(inp)
-    t0 = time.perf_counter()
-    r = O.fused_moe(d["x_bits"], d["wr_bits"], d["w13"], d["w2"], inp.shape.top_k, fp8=d["fp8"],
-                    w13_scale=d["w13_scale"], w2_scale=d["w2_scale"], grouped=oracle_grouped(inp),
-                    n_shared=inp.shape.n_shared)
-    return time.perf_counter() - t0, int((r["counts"] > 0).sum())
-
-
 class OracleSlices:
     """Bounded steps of the oracle.  A step runs the oracle's expert networks for one
     touched expert over all of its rows, restricted to a block of F intermediate features
@@ -296,9 +290,9 @@ def run_reference(args, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp64 (oracle; e4m3 codes decoded exactly)",
-        "data": "synthetic", "config": workload_config(s, "oracle"),
+        "data": "synthetic", "config": workload_config(s), "variant": "oracle",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
-                         "kind": "oracle",
+                         "kind": "oracle", "cores_available": len(os.sched_getaffinity(0)),
                          "sample": f"{args.steps} steps, each the expert networks of one "
                                    f"(touched expert, block of intermediate features) slice, "
                                    f"{len(sl.slices)} slices per layer over "
@@ -314,7 +308,12 @@ def run_reference(args, rank):
 
 # --------------------------------------------------------------------------- GPU arm
 
-def workload_config(s, variant):
+# Decode workloads measured beside the default (prefill) workload in the same run, so one
+# line covers both regimes of the metric: HBM-bound decode and tensor-bound prefill.
+EXTRA_WORKLOADS = (("mixtral_fp8_decode", 64), ("dsv3_fp8_decode", 256))
+
+
+def workload_config(s):
     weights = 3 * s.H * s.I * s.E_all * (1 if s.wdtype == "fp8" else 2)
     routing = "softmax top-k" if s.grouped is None else \
         (f"grouped sigmoid: {s.grouped[0]} groups, {s.grouped[1]} kept, "
@@ -323,65 +322,89 @@ def workload_config(s, variant):
     return {"workload": f"{s.name}: H={s.H} I={s.I} E={s.E}{shared} top_k={s.top_k} T={s.T} "
                         f"({s.wdtype} weights)",
             "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.top_k, "n_shared": s.n_shared,
-            "routing": routing, "variant": variant,
+            "routing": routing,
             "l2": f"inputs larger than L2: expert weights {weights / 1e9:.2f} GB vs "
                   f"{L2_BYTES / 2 ** 20:.0f} MB L2, no flush",
             "parallelism": "replicas (one independent layer per GPU)"}
 
 
-def run_ours(args, rank, world, local_rank):
+class Layer:
+    """Device tensors, descriptors and workspace of one workload."""
+
+    def __init__(self, s, dev, variant="auto", weights_on_device=False):
+        from mixture_experts_layer_26_b200 import capi
+        self.s, self.dev = s, dev
+        self.fp8 = s.wdtype == "fp8"
+        if weights_on_device:
+            # measurement only: the same distributions and per-expert quantisation drawn
+            # by the device's generator (the CPU draw of 11 GB takes about a minute)
+            x, wr = minp.make_activations(s, seed=0)
+            w13, w2, s13, s2 = minp.make_weights(s, seed=0, device=dev)
+            bias = minp.make_router_bias(s, seed=0)
+            self.inp = minp.MoEInputs(s, x, wr, w13, w2, s13, s2, bias)
+            self.weights_drawn = "on the device (torch CUDA generator, seed 0)"
+        else:
+            self.inp = minp.make_inputs(s, seed=0)
+            self.weights_drawn = "on the host (torch CPU generator, seed 0)"
+        inp = self.inp
+        self.x = inp.x.to(dev)
+        self.wr = inp.router_w.to(dev)
+        self.w13, self.w2 = inp.w13.to(dev), inp.w2.to(dev)
+        self.s13 = inp.w13_scale.to(dev) if self.fp8 else None
+        self.s2 = inp.w2_scale.to(dev) if self.fp8 else None
+        self.routing = routing_desc(inp, dev)
+        self.dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, self.fp8, variant,
+                                   routing=self.routing)
+        self.ws = capi.alloc_workspace(self.dims, dev)
+        self.sc = capi.make_scales(self.s13, self.s2)
+        self.out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device=dev)
+
+    def call(self, stream):
+        from mixture_experts_layer_26_b200 import capi
+        capi.fused_moe(self.dims, self.x, self.wr, self.w13, self.w2, self.sc, self.out,
+                       self.ws, stream)
+
+    def release(self):
+        for name in ("x", "wr", "w13", "w2", "s13", "s2", "ws", "out"):
+            setattr(self, name, None)
+        if self.inp is not None and self.inp.w13.is_cuda:
+            self.inp = None
+
+
+def measure_layer(L: Layer, args, dist, rank, world, dev, sample_clocks=True):
+    """Warm-up, exactly K timed steps (CUDA events on the launching stream, max over
+    ranks), then per-call events, a CUDA-graph replay, per-kernel events and the end-to-end
+    host-buffer call.  Returns the measured numbers (rank 0 reads them)."""
     from mixture_experts_layer_26_b200 import capi
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local_rank))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    s = minp.shape(args.workload, args.T)
-    fp8 = s.wdtype == "fp8"
-    inp = minp.make_inputs(s, seed=0)
-    x = inp.x.to(dev)
-    wr = inp.router_w.to(dev)
-    w13, w2 = inp.w13.to(dev), inp.w2.to(dev)
-    s13 = inp.w13_scale.to(dev) if fp8 else None
-    s2 = inp.w2_scale.to(dev) if fp8 else None
-    routing = routing_desc(inp, dev)
-    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, fp8, args.variant, routing=routing)
-    ws = capi.alloc_workspace(dims, dev)
-    sc = capi.make_scales(s13, s2)
-    out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device=dev)
+    s = L.s
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        return reduce_max(dist, v, dev)
-
     for _ in range(args.warmup):
-        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+        L.call(stream)
     torch.cuda.synchronize()
-    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+    assert capi.fused_moe_get_device_status(L.ws, stream) == capi.FMOE_OK
 
-    # ---- timed region: exactly K steps
+    # ---- timed region: exactly K steps.  The clock sampler runs from here through the
+    # per-call and per-kernel loops of the same workload (short timed regions would
+    # otherwise see one or two samples).
     barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(torch.cuda.get_device_properties(dev)) if rank == 0 else None
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev)) \
+        if (rank == 0 and sample_clocks) else None
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(args.steps):
-        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+        L.call(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    clocks = sampler.stop() if sampler is not None else None
-    ms = max_over_ranks(ev0.elapsed_time(ev1))
-    status = capi.fused_moe_get_device_status(ws, stream)
+    ms = reduce_max(dist, ev0.elapsed_time(ev1), dev)
+    status = capi.fused_moe_get_device_status(L.ws, stream)
     assert status == capi.FMOE_OK, capi.status_string(status)
-    ms_step = ms / args.steps
-    value = tokens_per_second(world, s.T, args.steps, ms)
 
     # ---- per-call distribution (events around every call) and a CUDA-graph replay of the
     # same call; both after the timed region, neither feeds `value`
@@ -390,7 +413,7 @@ def run_ours(args, rank, world, local_rank):
                for _ in range(n_calls)]
     for c0, c1 in call_ev:
         c0.record(stream)
-        capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, stream)
+        L.call(stream)
         c1.record(stream)
     torch.cuda.synchronize()
     per_call = sorted(c0.elapsed_time(c1) for c0, c1 in call_ev)
@@ -400,10 +423,10 @@ def run_ours(args, rank, world, local_rank):
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, side)  # warm-up on the side stream
+            L.call(side)  # warm-up on the side stream
         stream.wait_stream(side)
         with torch.cuda.graph(g, stream=side):
-            capi.fused_moe(dims, x, wr, w13, w2, sc, out, ws, side)
+            L.call(side)
         torch.cuda.synchronize()
         g.replay()
         torch.cuda.synchronize()
@@ -417,33 +440,34 @@ def run_ours(args, rank, world, local_rank):
         del g
     except RuntimeError as exc:  # capture unsupported in this environment: report, go on
         print(f"graph replay skipped: {exc}", file=sys.stderr)
-    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+    assert capi.fused_moe_get_device_status(L.ws, stream) == capi.FMOE_OK
 
     # ---- per-kernel times (events after every launch), same inputs, after the timed region
     nprof = max(5, min(args.steps, 200))
     per = {}
     for _ in range(nprof):
-        for name, t in capi.fused_moe_profile(dims, x, wr, w13, w2, sc, out, ws, stream):
+        for name, t in capi.fused_moe_profile(L.dims, L.x, L.wr, L.w13, L.w2, L.sc, L.out,
+                                              L.ws, stream):
             per.setdefault(name, []).append(t)
     kern_ms = {k: statistics.mean(v) for k, v in per.items()}
-    _, plan = capi.fused_moe_debug_scalars(ws, stream)
+    clocks = sampler.stop() if sampler is not None else None
+    _, plan = capi.fused_moe_debug_scalars(L.ws, stream)
 
     # ---- end to end through the host-buffer entry point
-    x_host = inp.x.clone().pin_memory()
+    x_host = L.inp.x.clone().pin_memory()
     out_host = torch.empty(s.T, s.H, dtype=torch.bfloat16).pin_memory()
     n_e2e = max(3, min(args.steps, 500))
     for _ in range(3):
-        capi.fused_moe_host_io(dims, x_host, wr, w13, w2, sc, out_host, ws, stream)
+        capi.fused_moe_host_io(L.dims, x_host, L.wr, L.w13, L.w2, L.sc, out_host, L.ws, stream)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(n_e2e):
-        capi.fused_moe_host_io(dims, x_host, wr, w13, w2, sc, out_host, ws, stream)
+        capi.fused_moe_host_io(L.dims, x_host, L.wr, L.w13, L.w2, L.sc, out_host, L.ws, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = tokens_per_second(world, s.T, n_e2e, e2e_ms)
+    e2e_ms = reduce_max(dist, e0.elapsed_time(e1), dev)
 
     # ---- experts the batch touched, from the GPU routing + permutation steps
     R = s.R
@@ -453,29 +477,93 @@ def run_ours(args, rank, world, local_rank):
     offs_d = torch.empty(s.E_all + 1, dtype=torch.int32, device=dev)
     rows_d = torch.empty(R, dtype=torch.int32, device=dev)
     inv_d = torch.empty(R, dtype=torch.int32, device=dev)
-    aperm_d = torch.empty(R, s.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
-    capi.fused_moe_route(dims, x, wr, ids_d, tw_d, ws, stream)
-    capi.fused_moe_permute(dims, ids_d, x, sc, counts_d, offs_d, rows_d, inv_d, aperm_d, ws, stream)
+    aperm_d = torch.empty(R, s.H, dtype=torch.uint8 if L.fp8 else torch.bfloat16, device=dev)
+    capi.fused_moe_route(L.dims, L.x, L.wr, ids_d, tw_d, L.ws, stream)
+    capi.fused_moe_permute(L.dims, ids_d, L.x, L.sc, counts_d, offs_d, rows_d, inv_d, aperm_d,
+                           L.ws, stream)
     touched = int((counts_d > 0).sum().item())
+    max_rows = int(counts_d.max().item())
+    return dict(ms=ms, ms_step=ms / args.steps, value=tokens_per_second(world, s.T, args.steps, ms),
+                per_call=per_call, n_calls=n_calls, graph_ms=graph_ms, kern_ms=kern_ms,
+                plan=plan, clocks=clocks, e2e_value=tokens_per_second(world, s.T, n_e2e, e2e_ms),
+                touched=touched, max_rows=max_rows,
+                launches=capi.fused_moe_launches_per_call(L.dims) * args.steps)
 
-    if dist is not None:
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
 
-    # ---- roofline of the dominant kernel
-    esz = 1 if fp8 else 2
-    peaks, peak_kind = load_peaks()
+def fp8_peak_probe(dev, burst_iters=10, sustained_s=4.0, n=8192):
+    """The FP8 dense tensor peak of this GPU, measured with the library GEMM:
+    torch._scaled_mm on e4m3 operands (n x n x n, unit scales, bf16 out).  Burst: the best
+    of `burst_iters` individually timed calls after warm-up.  Sustained: back-to-back calls
+    for about `sustained_s` seconds (the power cap settles in).  Returns TFLOP/s figures."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()  # column-major
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    flops = 2.0 * n * n * n
+
+    def mm():
+        return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    for _ in range(5):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(burst_iters):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    # sustained: batches of 50 calls until the time is spent
+    total_ms, calls = 0.0, 0
+    t_end = time.perf_counter() + sustained_s
+    while time.perf_counter() < t_end:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(50):
+            mm()
+        e1.record()
+        torch.cuda.synchronize()
+        total_ms += e0.elapsed_time(e1)
+        calls += 50
+    del a, b
+    return {"burst_tflops": round(flops / (best / 1e3) / 1e12, 1),
+            "sustained_tflops": round(flops * calls / (total_ms / 1e3) / 1e12, 1),
+            "how": f"torch._scaled_mm e4m3 {n}x{n}x{n}, unit per-tensor scales, bf16 out; "
+                   f"burst = best of {burst_iters} timed calls, sustained = {calls} "
+                   f"back-to-back calls over {total_ms / 1e3:.1f} s"}
+
+
+def tensor_peak(fp8: bool, peaks, peak_kind, probe):
+    """(TFLOP/s, description) of the burst tensor peak for a contraction timed per launch."""
+    if fp8 and "fp8_tflops" in peaks:
+        return float(peaks["fp8_tflops"]), f"{peak_kind}: MEASURED_PEAKS.json fp8_tflops (burst)"
+    if fp8 and probe is not None:
+        return probe["burst_tflops"], "measured in this run: FP8 burst (" + probe["how"] + ")"
+    if fp8:
+        return 2.0 * peaks["bf16_tflops"], (f"{peak_kind}: 2 x bf16_tflops (burst), the nominal "
+                                            "dense FP8/bf16 ratio 4.5/2.25 (no FP8 probe)")
+    return float(peaks["bf16_tflops"]), f"{peak_kind}: bf16_tflops (burst)"
+
+
+def roofline_of(s, m, peaks, peak_kind, probe, args_workload):
+    """Roofline of the dominant kernel plus the step's HBM and tensor figures."""
+    kern_ms = m["kern_ms"]
+    esz = 1 if s.wdtype == "fp8" else 2
+    fp8 = s.wdtype == "fp8"
     dom = max(kern_ms, key=kern_ms.get)
     names = "".join(kern_ms)
     variant = "swap_ab" if "swapab" in names else ("normal_pair" if "pair" in names else "normal")
+    touched = m["touched"]
     gemm1_bytes = touched * 2 * s.H * s.I * esz          # weights of the touched experts
     gemm2_bytes = touched * s.H * s.I * esz
     gemm1_flops = 4.0 * s.R * s.H * s.I                  # gate and up: 2 x (2 R H I)
     gemm2_flops = 2.0 * s.R * s.H * s.I
     kind = dom.split("_")[0]
     roof = None
-    traffic = profiled_traffic(dom, f"{args.workload}_T{s.T}")
+    traffic = profiled_traffic(dom, f"{args_workload}_T{s.T}")
     if variant == "swap_ab" and kind in ("gemm1", "gemm2"):
         dom_bytes = gemm1_bytes if kind == "gemm1" else gemm2_bytes
         ach = dom_bytes / (kern_ms[dom] / 1e3) / 1e9
@@ -483,55 +571,149 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": dom, "kernel_us": round(1e3 * kern_ms[dom], 2),
                 "algorithmic_bytes": dom_bytes,
-                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"}
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"
+                             if peak_kind == "measured" else
+                             "fallback 6650 GB/s (no MEASURED_PEAKS.json)"}
     elif kind in ("gemm1", "gemm2"):
         dom_flops = gemm1_flops if kind == "gemm1" else gemm2_flops
-        # a contraction timed inside a long back-to-back step: the sustained peak; FP8 is
-        # the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 = 2
-        ratio = 2.0 if fp8 else 1.0
-        peak = ratio * peaks["bf16_tflops_sustained"]
+        # a contraction timed per launch (events around it): the burst peak of its dtype
+        peak, how = tensor_peak(fp8, peaks, peak_kind, probe)
         ach = dom_flops / (kern_ms[dom] / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
                 "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": traffic,
                 "kernel": dom, "kernel_us": round(1e3 * kern_ms[dom], 2),
-                "algorithmic_flops": dom_flops,
-                "peak_kind": f"{peak_kind}: {'2 x ' if fp8 else ''}bf16_tflops_sustained "
-                             f"(burst: {ratio * peaks['bf16_tflops']:.0f} TFLOP/s)"}
+                "algorithmic_flops": dom_flops, "peak_kind": how}
     step_weight_bytes = gemm1_bytes + gemm2_bytes
     step_flops = gemm1_flops + gemm2_flops
-    # cpu baseline: the oracle on the whole batch, once
+    ms_step = m["ms_step"]
+    step_hbm = {"weight_bytes": step_weight_bytes,
+                "achieved_gbs": round(step_weight_bytes / (ms_step / 1e3) / 1e9, 1),
+                "frac": round(step_weight_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                "touched_experts": touched, "max_rows_per_expert": m["max_rows"]}
+    ach_t = step_flops / (ms_step / 1e3) / 1e12
+    peak_t, how_t = tensor_peak(fp8, peaks, peak_kind, probe)
+    step_tensor = {"flops": step_flops, "achieved_tflops": round(ach_t, 1),
+                   "frac": round(ach_t / peak_t, 4), "peak_tflops": round(peak_t, 1),
+                   "peak_kind": how_t}
+    return variant, roof, step_hbm, step_tensor
+
+
+def cpu_baseline_sample(inp, budget_s: float):
+    """The oracle as it stands on a bounded sample of the workload, on all host cores the
+    process may use and on one core: the routing, permutation and combine once, then
+    (touched expert, feature block) slices of the expert networks for about `budget_s`
+    seconds per setting, extrapolated to the whole layer (all slices)."""
+    import threadpoolctl
+    cores = len(os.sched_getaffinity(0))
+    res = {}
+    for label, limit in (("all", cores), ("one", 1)):
+        with threadpoolctl.threadpool_limits(limit, user_api="blas"):
+            sl = OracleSlices(inp)
+            sl.step()  # BLAS thread start-up
+            sl.i = 0
+            n, t0 = 0, time.perf_counter()
+            while (time.perf_counter() - t0 < budget_s or n == 0) and n < len(sl.slices):
+                sl.step()
+                n += 1
+            dt = time.perf_counter() - t0
+            layer_s = sl.fixed_s + sl.combine_seconds() + dt / n * len(sl.slices)
+            res[label] = (inp.shape.T / layer_s, n, len(sl.slices), layer_s, blas_threads())
+    v, n, total, layer_s, threads = res["all"]
+    v1, n1, _, layer_s1, _ = res["one"]
+    return {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "cores_available": cores, "value_1core": v1,
+            "sample": f"routing, permutation and combine of the T={inp.shape.T} batch once, then "
+                      f"{n} of the {total} (touched expert, feature block) slices of the expert "
+                      f"networks timed on {threads} BLAS threads ({n1} on 1 core), extrapolated "
+                      f"to all slices: one layer = {layer_s:.1f} s ({layer_s1:.1f} s on 1 core)"}
+
+
+def run_ours(args, rank, world, local_rank):
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = minp.shape(args.workload, args.T)
+    L = Layer(s, dev, args.variant)
+    m = measure_layer(L, args, dist, rank, world, dev)
+
+    # decode regimes beside the default prefill workload, measured the same way
+    extras = []
+    if args.workload == DEFAULT_WORKLOAD and args.T in (None, minp.shape(DEFAULT_WORKLOAD).T) \
+            and not args.no_extras:
+        L.release()
+        torch.cuda.empty_cache()
+        for wl, T in EXTRA_WORKLOADS:
+            se = minp.shape(wl, T)
+            Le = Layer(se, dev, "auto", weights_on_device=se.E_all * se.H * se.I > 2 ** 31)
+            me = measure_layer(Le, args, dist, rank, world, dev)
+            extras.append((se, Le.weights_drawn, me))
+            Le.release()
+            torch.cuda.empty_cache()
+
+    # the FP8 tensor peak of this GPU (after the timed regions, so that they do not run on
+    # a GPU the probe has just heated)
+    probe = fp8_peak_probe(dev) if (rank == 0 and not args.no_peak_probe) else None
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    variant, roof, step_hbm, step_tensor = roofline_of(s, m, peaks, peak_kind, probe,
+                                                       args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        secs, _ = oracle_full_pass(inp)
-        cpu = {"value": s.T / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"one full oracle pass over the T={s.T} batch ({secs:.1f} s)"}
+        cpu = cpu_baseline_sample(L.inp, args.cpu_budget)
+    fp8 = s.wdtype == "fp8"
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "metric": METRIC, "value": round(m["value"], 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(m["ms_step"], 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
         "data": "synthetic (seeded; N(0,1) x, N(0,1/sqrt(fan_in)) weights, per-expert e4m3 scales)",
-        "config": workload_config(s, variant),
+        "config": workload_config(s),
+        "variant": variant,
         "roofline": roof,
-        "step_hbm": {"weight_bytes": step_weight_bytes,
-                     "achieved_gbs": round(step_weight_bytes / (ms_step / 1e3) / 1e9, 1),
-                     "frac": round(step_weight_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
-                     "touched_experts": touched},
-        "step_tensor": {"flops": step_flops,
-                        "achieved_tflops": round(step_flops / (ms_step / 1e3) / 1e12, 1)},
-        "kernels_us": {k: round(1e3 * v, 2) for k, v in kern_ms.items()},
-        "plan": plan,
+        "step_hbm": step_hbm,
+        "step_tensor": step_tensor,
+        "kernels_us": {k: round(1e3 * v, 2) for k, v in m["kern_ms"].items()},
+        "plan": m["plan"],
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+        "e2e": {"value": round(m["e2e_value"], 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": s.T * s.H * 2, "d2h_bytes_per_step": s.T * s.H * 2,
                 "api": "fused_moe_host_io (pinned host x and out)"},
-        "gpu_launches": capi.fused_moe_launches_per_call(dims) * args.steps,
-        "clocks": clocks,
-        "per_call_ms": {"calls": n_calls, "median": round(statistics.median(per_call), 5),
-                        "p95": round(per_call[min(n_calls - 1, int(0.95 * n_calls))], 5),
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
+        "per_call_ms": {"calls": m["n_calls"], "median": round(statistics.median(m["per_call"]), 5),
+                        "p95": round(m["per_call"][min(m["n_calls"] - 1, int(0.95 * m["n_calls"]))], 5),
                         "note": "events around each call, after the timed region"},
-        "graph_replay_ms_per_call": None if graph_ms is None else round(graph_ms, 5),
+        "graph_replay_ms_per_call": None if m["graph_ms"] is None else round(m["graph_ms"], 5),
+        "fp8_peak_probe": probe,
+        "hbm_peak": {"gbs": peaks["hbm_gbs"], "kind": peak_kind},
     }
+    if extras:
+        line["decode"] = []
+        for se, drawn, me in extras:
+            v_e, roof_e, hbm_e, ten_e = roofline_of(se, me, peaks, peak_kind, probe, se.name)
+            line["decode"].append({
+                "config": workload_config(se), "weights_drawn": drawn, "variant": v_e,
+                "value": round(me["value"], 1), "unit": "tokens/s", "steps": args.steps,
+                "ms_per_step": round(me["ms_step"], 5), "roofline": roof_e, "step_hbm": hbm_e,
+                "step_tensor": ten_e,
+                "kernels_us": {k: round(1e3 * v, 2) for k, v in me["kern_ms"].items()},
+                "e2e": {"value": round(me["e2e_value"], 1), "unit": "tokens/s",
+                        "h2d_bytes_per_step": se.T * se.H * 2,
+                        "d2h_bytes_per_step": se.T * se.H * 2,
+                        "api": "fused_moe_host_io (pinned host x and out)"},
+                "gpu_launches": me["launches"], "clocks": me["clocks"],
+                "per_call_ms": {"median": round(statistics.median(me["per_call"]), 5)},
+                "graph_replay_ms_per_call": None if me["graph_ms"] is None else round(me["graph_ms"], 5),
+            })
     print(json.dumps(line))
     return 0
 
@@ -730,12 +912,18 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral_fp8_decode",
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(minp.WORKLOADS) + sorted(minp.ROPE_WORKLOADS))
     ap.add_argument("--T", type=int, default=None,
-                    help="tokens (default: the workload's largest; 64 for the default workload)")
+                    help="tokens (default: the workload's largest; 4096 for the default workload)")
     ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal", "normal_pair"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the decode workloads measured beside the default one")
+    ap.add_argument("--no-peak-probe", action="store_true",
+                    help="skip the FP8 tensor-peak probe (torch._scaled_mm)")
+    ap.add_argument("--cpu-budget", type=float, default=8.0,
+                    help="seconds of oracle expert work per core setting in cpu_baseline")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

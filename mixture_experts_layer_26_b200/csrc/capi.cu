@@ -555,6 +555,21 @@ fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const
 
 }  // namespace
 
+namespace fmoe {
+// The argument checks of the one-call layer, in the order fused_moe runs them: dims,
+// then (T > 0) the tensor pointers and the FP8 weight scales.  No CUDA call.
+fmoe_status check_layer_args(const fmoe_dims* dims, const void* x, const void* router_w,
+                             const void* w13, const void* w2, const fmoe_scales* scales,
+                             const void* out) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, router_w, w13, w2, out));
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  return FMOE_OK;
+}
+}  // namespace fmoe
+
 // ------------------------------------------------------------------ public API
 
 extern "C" {
@@ -638,11 +653,8 @@ fmoe_status fused_moe_combine(const fmoe_dims* dims, const float* y_perm, const 
 fmoe_status fused_moe(const fmoe_dims* dims, const void* x, const void* router_w, const void* w13,
                       const void* w2, const fmoe_scales* scales, void* out, void* ws,
                       size_t ws_bytes, fmoe_stream stream) {
-  FMOE_TRY(check_dims(dims));
+  FMOE_TRY(fmoe::check_layer_args(dims, x, router_w, w13, w2, scales, out));
   if (dims->T == 0) return FMOE_OK;
-  FMOE_TRY(check_ptrs(x, router_w, w13, w2, out));
-  FMOE_TRY(check_fp8_scales(*dims, scales));
-  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
   const Layout L = make_layout(*dims);
   FMOE_TRY(check_ws(L, ws, ws_bytes));
   return fused_impl(*dims, L, x, router_w, w13, w2, scales, out, static_cast<char*>(ws),

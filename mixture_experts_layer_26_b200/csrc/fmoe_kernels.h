@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "fmoe_common.cuh"
+#include "fused_moe.h"
 
 namespace fmoe {
 
@@ -222,6 +223,13 @@ struct CombineArgs {
   int T, H, k;
 };
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- host checks
+// The argument checks fused_moe runs before any CUDA call (capi.cu): dims, then for
+// T > 0 the tensor pointers (non-null, 16-byte aligned) and the FP8 weight scales.
+fmoe_status check_layer_args(const fmoe_dims* dims, const void* x, const void* router_w,
+                             const void* w13, const void* w2, const fmoe_scales* scales,
+                             const void* out);
 
 // ----------------------------------------------------------------------------- inverse RoPE
 struct RopeArgs {

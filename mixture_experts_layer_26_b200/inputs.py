@@ -90,8 +90,8 @@ def shape(workload: str, T: Optional[int] = None) -> MoEShape:
     return MoEShape(T=T, name=workload, **w)
 
 
-def _gen(seed: int, tag: int, index: int = 0) -> torch.Generator:
-    g = torch.Generator()
+def _gen(seed: int, tag: int, index: int = 0, device=None) -> torch.Generator:
+    g = torch.Generator() if device is None else torch.Generator(device=device)
     g.manual_seed((seed * 1_000_003 + tag * 10_007 + index) & 0x7FFF_FFFF_FFFF_FFFF)
     return g
 
@@ -99,7 +99,7 @@ def _gen(seed: int, tag: int, index: int = 0) -> torch.Generator:
 def _to_e4m3(w: torch.Tensor):
     """Per-tensor scale and e4m3fn bytes of one fp32 expert tensor (torch's cast)."""
     amax = w.abs().max().to(torch.float32)
-    sw = (amax / E4M3_MAX) if amax > 0 else torch.tensor(1.0)
+    sw = (amax / E4M3_MAX) if amax > 0 else torch.tensor(1.0, device=w.device)
     q = torch.clamp(w / sw, -E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
     return float(sw), q.view(torch.uint8)
 
@@ -134,18 +134,26 @@ def make_activations(s: MoEShape, seed: int = 0, T: Optional[int] = None):
     return x.to(torch.bfloat16), wr.to(torch.bfloat16)
 
 
-def make_weights(s: MoEShape, seed: int = 0):
-    """Expert weights in the layer's storage format, generated one expert at a time."""
+def make_weights(s: MoEShape, seed: int = 0, device=None):
+    """Expert weights in the layer's storage format, generated one expert at a time.
+
+    device=None draws on the host (the bytes every parity check uses).  A CUDA device
+    draws there with the device's generator, seeded the same way: the same distributions
+    and per-expert quantisation but a different random stream, for measurements whose
+    weights are too large to draw on the host quickly (the routing depends only on x and
+    router_w, which stay host-drawn)."""
     fp8 = s.wdtype == "fp8"
     dt = torch.uint8 if fp8 else torch.bfloat16
-    w13 = torch.empty(s.E_all, 2 * s.I, s.H, dtype=dt)
-    w2 = torch.empty(s.E_all, s.H, s.I, dtype=dt)
+    w13 = torch.empty(s.E_all, 2 * s.I, s.H, dtype=dt, device=device)
+    w2 = torch.empty(s.E_all, s.H, s.I, dtype=dt, device=device)
     s13 = torch.ones(s.E_all, dtype=torch.float32)
     s2 = torch.ones(s.E_all, dtype=torch.float32)
     for e in range(s.E_all):
-        a = torch.randn(2 * s.I, s.H, generator=_gen(seed, 3, e), dtype=torch.float32)
+        a = torch.randn(2 * s.I, s.H, generator=_gen(seed, 3, e, device), dtype=torch.float32,
+                        device=device)
         a *= 1.0 / math.sqrt(s.H)
-        b = torch.randn(s.H, s.I, generator=_gen(seed, 4, e), dtype=torch.float32)
+        b = torch.randn(s.H, s.I, generator=_gen(seed, 4, e, device), dtype=torch.float32,
+                        device=device)
         b *= 1.0 / math.sqrt(s.I)
         if fp8:
             s13[e], w13[e] = _to_e4m3(a)

@@ -288,3 +288,35 @@ def test_host_properties_over_many_dims():
         kw = dict(T=4, H=256, I=128, E=8, k=2)
         kw.update(bad)
         assert capi.workspace_size(capi.make_dims(kw["T"], kw["H"], kw["I"], kw["E"], kw["k"], True)) == 0
+
+
+def call_static(d, x=FAKE, rw=FAKE, w13=FAKE, w2=FAKE, out=FAKE, status=None, scales=True):
+    sc = capi.FmoeScales(FAKE, FAKE, 0.0, 0.0) if scales else None
+    return capi.fused_moe_static_workspace(d, _T(x), _T(rw), _T(w13), _T(w2), sc, _T(out),
+                                           None if status is None else _T(status), stream=0,
+                                           check=False)
+
+
+def test_static_workspace_checks_arguments_before_any_cuda_call():
+    """fused_moe_static_workspace returns fused_moe's own status codes for bad arguments,
+    and the size limit, before any CUDA call: on a machine without a GPU every one of
+    these returns its code instead of FMOE_ERR_CUDA."""
+    assert call_static(dims(), x=0) == capi.FMOE_ERR_INVALID_ARG
+    assert call_static(dims(), out=0) == capi.FMOE_ERR_INVALID_ARG
+    assert call_static(dims(), w2=FAKE + 8) == capi.FMOE_ERR_UNSUPPORTED   # misaligned
+    assert call_static(dims(), scales=False) == capi.FMOE_ERR_INVALID_ARG  # FP8 needs scales
+    assert call_static(dims(k=9)) == capi.FMOE_ERR_INVALID_ARG
+    assert call_static(dims(H=384)) == capi.FMOE_ERR_UNSUPPORTED           # H % 256 != 0
+    assert call_static(dims(), status=FAKE + 2) == capi.FMOE_ERR_UNSUPPORTED
+    # dims whose workspace exceeds the 64 MiB array (Mixtral-like FP8 decode at T = 64)
+    big = dims(T=64, H=4096, I=14336)
+    assert capi.workspace_size(big) > capi.STATIC_WS_BYTES
+    assert call_static(big) == capi.FMOE_ERR_WORKSPACE
+    assert call_static(dims(T=0)) == capi.FMOE_OK  # no tokens: nothing to do
+
+
+@pytest.mark.skipif(capi is not None and __import__("torch").cuda.is_available(),
+                    reason="checks the no-GPU behaviour")
+def test_static_workspace_valid_arguments_reach_cuda():
+    # valid arguments pass every check and only then meet the missing GPU
+    assert call_static(dims()) == capi.FMOE_ERR_CUDA
