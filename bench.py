@@ -718,6 +718,98 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_tp_ours(args, rank, world, local_rank):
+    """Tensor parallelism over the intermediate features: rank r of N holds shard r of
+    every expert and the N ranks compute ONE batch together (strong scaling).  A step is
+    one layer call: begin (route, permute, first contraction), all-reduce MAX of max |h|,
+    end (second contraction, fp32 partial output), all-reduce SUM of the partial outputs,
+    finish (bf16).  With N = 1 the collectives are skipped (a group of one)."""
+    from mixture_experts_layer_26_b200 import capi, tp
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = minp.shape(args.workload, args.T)
+    fp8 = s.wdtype == "fp8"
+    inp = minp.make_inputs(s, seed=0)
+    w13_r, w2_r = tp.shard_weights(inp.w13, inp.w2, rank, world)
+    x = inp.x.to(dev)
+    ident = (lambda t: t) if dist is None else None
+    layer = tp.TensorParallelMoE(inp.router_w.to(dev), w13_r.to(dev), w2_r.to(dev), s.top_k,
+                                 inp.w13_scale.to(dev) if fp8 else None,
+                                 inp.w2_scale.to(dev) if fp8 else None,
+                                 routing=routing_desc(inp, dev), variant=args.variant,
+                                 reduce_max=ident, reduce_sum=ident)
+    out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer(x, out, stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev)) if rank == 0 else None
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        layer(x, out, stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    ms = reduce_max(dist, ev0.elapsed_time(ev1), dev)
+    ws = next(iter(layer._bufs.values()))[0]
+    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+    # end to end: x from pinned host memory, out back to pinned host memory, every step
+    x_host = inp.x.clone().pin_memory()
+    out_host = torch.empty(s.T, s.H, dtype=torch.bfloat16).pin_memory()
+    n_e2e = max(3, min(args.steps, 200))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        x.copy_(x_host, non_blocking=True)
+        layer(x, out, stream)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(dist, e0.elapsed_time(e1), dev)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    ms_step = ms / args.steps
+    cfg = workload_config(s)
+    cfg["parallelism"] = f"tensor parallel over the intermediate features: {world} shard(s) " \
+                         f"of I/{world} = {s.I // world}, NCCL all-reduce of max|h| and of the " \
+                         "fp32 partial output"
+    line = {
+        "metric": METRIC, "value": round(s.T * args.steps / (ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16 (fp32 accumulate)",
+        "data": "synthetic (seeded; N(0,1) x, N(0,1/sqrt(fan_in)) weights, per-expert e4m3 scales)",
+        "config": cfg, "variant": f"tp{world}",
+        "e2e": {"value": round(s.T * n_e2e / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": s.T * s.H * 2, "d2h_bytes_per_step": s.T * s.H * 2,
+                "api": "TensorParallelMoE with pinned host copies of x and out"},
+        # the one-call kernels plus amax_reduce and the bf16 finish, per step
+        "gpu_launches": (capi.fused_moe_launches_per_call(layer.dims(s.T)) + 2) * args.steps,
+        "clocks": clocks, "cpu_baseline": None,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 # --------------------------------------------------------------------------- inverse RoPE
 
 ROPE_METRIC = ("inverse-RoPE + per-head FP8 quantisation tokens/s; achieved HBM GB/s vs peak")
@@ -918,6 +1010,8 @@ def main(argv=None):
                     help="tokens (default: the workload's largest; 4096 for the default workload)")
     ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal", "normal_pair"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallelism: the ranks share one layer, each holding I/N")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the decode workloads measured beside the default one")
     ap.add_argument("--no-peak-probe", action="store_true",
@@ -936,6 +1030,8 @@ def main(argv=None):
         return run_rope_ours(args, rank, world, local_rank)
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.tp:
+        return run_tp_ours(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 

@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define FUSED_MOE_ABI_VERSION 3
+#define FUSED_MOE_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define FMOE_API __attribute__((visibility("default")))
@@ -233,6 +233,50 @@ FMOE_API fmoe_status fused_moe(const fmoe_dims* dims, const void* x, const void*
 FMOE_API fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host, const void* router_w,
                               const void* w13, const void* w2, const fmoe_scales* scales,
                               void* out_host, void* ws, size_t ws_bytes, fmoe_stream stream);
+
+/* ---------------------------------------------------------------------------------
+ * Tensor parallelism over the intermediate dimension (N shards).
+ *
+ * The pages measure their serving result at 8-way tensor parallelism (agentic-affairs.com,
+ * third change; modelsatwork.news, "The three changes", recompilation) and note that on
+ * multi-GPU setups every GPU waits when one of them stalls (codebridge-ai.com blog
+ * "AWS MoE kernel: WGMMA, Triton, TTFT", section 3).  The layer splits over the expert
+ * intermediate features: shard r of N holds, for every expert, features
+ * [r*I/N, (r+1)*I/N) -- those rows of W1 and of W3, and those columns of W2 -- so
+ *   w13_r [E, 2*I/N, H]: rows 0..I/N-1 = W1 rows r*I/N.., rows I/N.. = W3 rows r*I/N..
+ *   w2_r  [E, H, I/N]:   W2[:, :, r*I/N : (r+1)*I/N]
+ * with the unsharded per-expert FP8 scales (the bytes are slices of the same tensors).
+ * Routing and the activation quantisation are computed identically on every shard.  Each
+ * shard's h is a slice of the unsharded h, and the per-tensor scale of h needs the max
+ * over all of it, so a shard's call is split around one cross-shard exchange:
+ *   1. fused_moe_tp_begin    route, permute, first contraction; writes this shard's
+ *                            max |h| to amax_h (one fp32 device word)
+ *   2. the caller reduces amax_h with MAX over the shards (e.g. NCCL all-reduce)
+ *   3. fused_moe_tp_end      quantises h with the shards' max, second contraction and
+ *                            combine into this shard's fp32 partial output [T, H]
+ *   4. the caller reduces the partial outputs with SUM over the shards
+ *   5. fused_moe_tp_finish   out = bf16(sum), round to nearest even
+ * The result is the unsharded layer's up to fp32 summation order: the e4m3 codes of h
+ * are the unsharded ones.  dims.I is the shard's I/N (a multiple of 128); the workspace
+ * is sized by fused_moe_workspace_size(dims) and carries state from step 1 to step 3, so
+ * use the same ws for both.  With one shard the five steps equal fused_moe.
+ * T == 0 launches nothing (amax_h is not written).  The same checks and status codes as
+ * fused_moe apply, and amax_h must be non-null and 4-byte aligned. */
+FMOE_API fmoe_status fused_moe_tp_begin(const fmoe_dims* dims, const void* x, const void* router_w,
+                                        const void* w13, const fmoe_scales* scales, float* amax_h,
+                                        void* ws, size_t ws_bytes, fmoe_stream stream);
+
+/* Step 3.  amax_h: device word holding the max of every shard's step-1 value (ignored in
+ * the bf16 format and when scales->a2_scale > 0); out_partial [T, H] fp32 device out:
+ * this shard's sum over the K slots of each token, before any rounding to bf16. */
+FMOE_API fmoe_status fused_moe_tp_end(const fmoe_dims* dims, const void* w2, const fmoe_scales* scales,
+                                      const float* amax_h, float* out_partial, void* ws,
+                                      size_t ws_bytes, fmoe_stream stream);
+
+/* Step 5.  out_sum [n] fp32, out [n] bf16 (device, 16-byte aligned); n a multiple of 8
+ * (T*H always is).  Asynchronous on `stream`. */
+FMOE_API fmoe_status fused_moe_tp_finish(int64_t n, const float* out_sum, void* out,
+                                         fmoe_stream stream);
 
 /* Number of kernels one fused_moe call launches for these dims: router, gemm1,
  * finalize1 (SWAP_AB only), quant_h (FP8 only), gemm2 and combine, plus permute and

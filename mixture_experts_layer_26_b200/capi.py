@@ -37,7 +37,8 @@ EXPORTED = (
     "fused_moe_combine", "fused_moe", "fused_moe_host_io", "fused_moe_get_device_status",
     "fused_moe_debug_scalars", "fused_moe_launches_per_call", "fused_moe_profile",
     "fused_moe_static_workspace", "fused_moe_selftest_wait",
-    "fused_inv_rope_fp8_quant_per_head",
+    "fused_inv_rope_fp8_quant_per_head", "fused_moe_tp_begin", "fused_moe_tp_end",
+    "fused_moe_tp_finish",
 )
 STATIC_WS_BYTES = 64 << 20  # FUSED_MOE_STATIC_WS_BYTES
 
@@ -103,6 +104,13 @@ _inv_rope = _sig("fused_inv_rope_fp8_quant_per_head", c_int32, POINTER(FmoeRopeD
 _profile = _sig("fused_moe_profile", c_int32, _DP, c_void_p, c_void_p, c_void_p, c_void_p, _SP,
                 c_void_p, c_void_p, c_size_t, c_void_p, POINTER(c_float), POINTER(c_char_p),
                 c_int32, POINTER(c_int32))
+
+
+_tp_begin = _sig("fused_moe_tp_begin", c_int32, _DP, c_void_p, c_void_p, c_void_p, _SP, c_void_p,
+                 c_void_p, c_size_t, c_void_p)
+_tp_end = _sig("fused_moe_tp_end", c_int32, _DP, c_void_p, _SP, c_void_p, c_void_p, c_void_p,
+               c_size_t, c_void_p)
+_tp_finish = _sig("fused_moe_tp_finish", c_int32, ctypes.c_int64, c_void_p, c_void_p, c_void_p)
 
 
 class FusedMoEError(RuntimeError):
@@ -238,6 +246,31 @@ def fused_moe_host_io(dims, x_host, router_w, w13, w2, scales, out_host, ws, str
     st = _host_io(ctypes.byref(dims), _ptr(x_host), _ptr(router_w), _ptr(w13), _ptr(w2), sp,
                   _ptr(out_host), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
     return _check(st, "fused_moe_host_io") if check else st
+
+
+def fused_moe_tp_begin(dims, x, router_w, w13, scales, amax_h, ws, stream=None, check=True) -> int:
+    """Tensor-parallel shard, step 1: route, permute and the first contraction on this
+    shard's w13; writes the shard's max |h| into amax_h (one fp32 device word)."""
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _tp_begin(ctypes.byref(dims), _ptr(x), _ptr(router_w), _ptr(w13), sp, _ptr(amax_h),
+                   _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_tp_begin") if check else st
+
+
+def fused_moe_tp_end(dims, w2, scales, amax_h, out_partial, ws, stream=None, check=True) -> int:
+    """Tensor-parallel shard, step 3: with amax_h holding the max over all shards, the
+    second contraction and combine into this shard's fp32 partial output [T, H]."""
+    sp = ctypes.byref(scales) if scales is not None else None
+    st = _tp_end(ctypes.byref(dims), _ptr(w2), sp, _ptr(amax_h), _ptr(out_partial), _ptr(ws),
+                 ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "fused_moe_tp_end") if check else st
+
+
+def fused_moe_tp_finish(out_sum, out, stream=None, check=True) -> int:
+    """Tensor-parallel step 5: out (bf16) = round(out_sum (fp32)), element by element."""
+    n = out_sum.numel() if out_sum is not None else 0
+    st = _tp_finish(n, _ptr(out_sum), _ptr(out), _stream(stream))
+    return _check(st, "fused_moe_tp_finish") if check else st
 
 
 def fused_moe_get_device_status(ws, stream=None) -> int:

@@ -368,21 +368,37 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   return FMOE_OK;
 }
 
-// Steps a3-a4.  plan_done: the permute launch already wrote the GEMM plan.  fused_out
-// (one-call path): in the swap-AB variant finish the second contraction's partials
-// straight into the combined output (needs ids and inv) instead of writing y.
-fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm,
-                         const int32_t* offsets, const int32_t* rows, const float* tw,
-                         const void* w13, const void* w2, const fmoe_scales* sc, float* y,
-                         char* W, cudaStream_t s, bool plan_done = false,
-                         void* fused_out = nullptr, const int32_t* ids = nullptr,
-                         const int32_t* inv = nullptr, bool plan_two_back = false) {
+// The grouped-GEMM arguments both contractions share.
+GemmArgs gemm_base(const Layout& L, const int32_t* rows, const float* tw, char* W,
+                   const fmoe_dims& d) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+  GemmArgs g{};
+  g.chunks = reinterpret_cast<Chunk*>(W + L.chunks);
+  g.hdr = hdr;
+  g.hdr_w = hdr;
+  g.status = &hdr->status;
+  g.topk_w = tw;
+  g.sorted_rows = rows;
+  g.amax_part = reinterpret_cast<float*>(W + L.amax_h);
+  g.R = L.R;
+  g.I = d.I;
+  g.H = d.H;
+  g.chunk_rows = L.chunk_rows;
+  g.nstages = gemm_stages(L.swap, L.chunk_rows);
+  g.wait_budget_ns = kWaitBudgetNs;
+  return g;
+}
+
+// Step a3: plan (unless the permutation launch wrote it), the first contraction with
+// SiLU(g)*u, and (swap-AB) the split-K finish of h with its max partials.
+fmoe_status experts_first(const fmoe_dims& d, const Layout& L, const void* a_perm,
+                          const int32_t* offsets, const int32_t* rows, const float* tw,
+                          const void* w13, const fmoe_scales* sc, char* W, cudaStream_t s,
+                          bool plan_done, bool plan_two_back) {
   const int sms = num_sms();
   const bool fp8 = L.fp8, swap = L.swap;
   const int H = d.H, I = d.I, E = experts_all(d), R = L.R;
-  const int bk = fp8 ? 128 : 64;
   WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
-  Chunk* chunks = reinterpret_cast<Chunk*>(W + L.chunks);
   float* amax_h = reinterpret_cast<float*>(W + L.amax_h);
   float* hbuf = reinterpret_cast<float*>(W + L.h);
   void* hq = W + L.hq;
@@ -398,34 +414,21 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   }
 
   const uint32_t xbox = swap ? 16u : 128u;
-  GemmArgs g{};
+  GemmArgs g = gemm_base(L, rows, tw, W, d);
   if (!encode_map(&g.map_w, w13, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(E) * 2 * I,
                   swap ? 16u : 128u) ||
       !encode_map(&g.map_x, a_perm, fp8, static_cast<uint64_t>(H), static_cast<uint64_t>(R), xbox))
     return FMOE_ERR_CUDA;
-  g.chunks = chunks;
-  g.hdr = hdr;
-  g.hdr_w = hdr;
-  g.status = &hdr->status;
   g.out = swap ? reinterpret_cast<float*>(W + L.p1) : (fp8 ? hbuf : nullptr);
   g.out_bf16 = fp8 ? nullptr : static_cast<uint16_t*>(hq);
   g.h_out = fp8 ? hbuf : nullptr;
   g.w_scale = fp8 ? sc->w13_scale : nullptr;
-  g.topk_w = tw;
-  g.sorted_rows = rows;
-  g.amax_part = amax_h;
-  g.R = R;
   g.K = H;
   g.Nout = 2 * I;
-  g.I = I;
-  g.H = H;
   g.rows_per_expert = 2 * I;
-  g.chunk_rows = L.chunk_rows;
-  g.nstages = gemm_stages(swap, L.chunk_rows);
   // the first contraction may prefetch weights when its plan came two launches back (the
-  // gather ran in between); the second one always may (gemm1 at least sits in between)
+  // gather ran in between)
   g.prefetch_w = plan_two_back ? 1 : 0;
-  g.wait_budget_ns = kWaitBudgetNs;
   if (L.pair)
     FMOE_LAUNCH("gemm1_pair", launch_gemm_pair(g, fp8, 1, sms, s), s);
   else
@@ -447,12 +450,34 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
     f.fp8 = fp8 ? 1 : 0;
     FMOE_LAUNCH("finalize1", launch_finalize1(f, sms, s), s);
   }
+  return FMOE_OK;
+}
+
+// Step a4 (and, swap-AB, the finish of the output): FP8 re-quantisation of h (its max
+// from this call's partials, or from amax_in), the second contraction, then either the
+// combined output (fused_out bf16 or out_f32 fp32 sums, swap-AB: split-K partials
+// finished and combined in one pass) or y (finalize2 for swap-AB; the normal variants'
+// GEMM writes y itself and the caller combines).
+fmoe_status experts_second(const fmoe_dims& d, const Layout& L, const int32_t* offsets,
+                           const int32_t* rows, const float* tw, const void* w2,
+                           const fmoe_scales* sc, float* y, char* W, cudaStream_t s,
+                           void* fused_out, float* out_f32, const int32_t* ids,
+                           const int32_t* inv, const float* amax_in) {
+  const int sms = num_sms();
+  const bool fp8 = L.fp8, swap = L.swap;
+  const int H = d.H, I = d.I, E = experts_all(d), R = L.R;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
+  float* amax_h = reinterpret_cast<float*>(W + L.amax_h);
+  float* hbuf = reinterpret_cast<float*>(W + L.h);
+  void* hq = W + L.hq;
+
   if (fp8) {
     QuantHArgs q{};
     q.h = hbuf;
     q.h_bf16 = nullptr;
     q.hq = static_cast<uint8_t*>(hq);
     q.amax_part = amax_h;
+    q.amax_in = amax_in;
     q.hdr = hdr;
     q.R = R;
     q.I = I;
@@ -460,7 +485,8 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
     FMOE_LAUNCH("quant_h", launch_quant_h(q, sms, s), s);
   }
 
-  GemmArgs g2 = g;
+  const uint32_t xbox = swap ? 16u : 128u;
+  GemmArgs g2 = gemm_base(L, rows, tw, W, d);
   if (!encode_map(&g2.map_w, w2, fp8, static_cast<uint64_t>(I), static_cast<uint64_t>(E) * H, 128) ||
       !encode_map(&g2.map_x, hq, fp8, static_cast<uint64_t>(I), static_cast<uint64_t>(R), xbox))
     return FMOE_ERR_CUDA;
@@ -471,13 +497,13 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   g2.K = I;
   g2.Nout = H;
   g2.rows_per_expert = H;
-  g2.prefetch_w = 1;
+  g2.prefetch_w = 1;  // the chunk list was written at least two launches back (gemm1 between)
   if (L.pair)
     FMOE_LAUNCH("gemm2_pair", launch_gemm_pair(g2, fp8, 2, sms, s), s);
   else
     FMOE_LAUNCH(swap ? "gemm2_swapab" : "gemm2_normal", launch_gemm(g2, fp8, swap, 2, sms, s), s);
 
-  if (swap && fused_out != nullptr) {
+  if (swap && (fused_out != nullptr || out_f32 != nullptr)) {
     CombinePartialsArgs c{};
     c.part = reinterpret_cast<const float*>(W + L.p2);
     c.inv_perm = inv;
@@ -486,6 +512,7 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
     c.w2_scale = fp8 ? sc->w2_scale : nullptr;
     c.hdr = hdr;
     c.out = static_cast<uint16_t*>(fused_out);
+    c.out_f32 = out_f32;
     c.T = d.T;
     c.H = H;
     c.k = slots_of(d);
@@ -511,12 +538,27 @@ fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm
   return FMOE_OK;
 }
 
+// Steps a3-a4.  plan_done: the permute launch already wrote the GEMM plan.  fused_out
+// (one-call path): in the swap-AB variant finish the second contraction's partials
+// straight into the combined output (needs ids and inv) instead of writing y.
+fmoe_status experts_impl(const fmoe_dims& d, const Layout& L, const void* a_perm,
+                         const int32_t* offsets, const int32_t* rows, const float* tw,
+                         const void* w13, const void* w2, const fmoe_scales* sc, float* y,
+                         char* W, cudaStream_t s, bool plan_done = false,
+                         void* fused_out = nullptr, const int32_t* ids = nullptr,
+                         const int32_t* inv = nullptr, bool plan_two_back = false) {
+  FMOE_TRY(experts_first(d, L, a_perm, offsets, rows, tw, w13, sc, W, s, plan_done, plan_two_back));
+  return experts_second(d, L, offsets, rows, tw, w2, sc, y, W, s, fused_out, nullptr, ids, inv,
+                        nullptr);
+}
+
 fmoe_status combine_impl(const fmoe_dims& d, const float* y, const int32_t* inv, void* out,
-                         cudaStream_t s) {
+                         cudaStream_t s, float* out_f32 = nullptr) {
   CombineArgs c{};
   c.y = y;
   c.inv_perm = inv;
   c.out = static_cast<uint16_t*>(out);
+  c.out_f32 = out_f32;
   c.T = d.T;
   c.H = d.H;
   c.k = slots_of(d);
@@ -524,33 +566,58 @@ fmoe_status combine_impl(const fmoe_dims& d, const float* y, const int32_t* inv,
   return FMOE_OK;
 }
 
-fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
-                       const void* w13, const void* w2, const fmoe_scales* sc, void* out, char* W,
+// Workspace views of the one-call path's routing buffers and y.
+struct OneCall {
+  int32_t *ids, *counts, *offsets, *rows, *inv;
+  float *tw, *y;
+  OneCall(const Layout& L, char* W)
+      : ids(reinterpret_cast<int32_t*>(W + L.ids)),
+        counts(reinterpret_cast<int32_t*>(W + L.counts)),
+        offsets(reinterpret_cast<int32_t*>(W + L.offsets)),
+        rows(reinterpret_cast<int32_t*>(W + L.rows)),
+        inv(reinterpret_cast<int32_t*>(W + L.inv)),
+        tw(reinterpret_cast<float*>(W + L.tw)),
+        y(reinterpret_cast<float*>(W + L.y)) {}
+};
+
+// Steps a1-a2 of the one-call path, then a3 (the first contraction).
+fmoe_status first_half(const fmoe_dims& d, const Layout& L, const OneCall& b, const void* x,
+                       const void* rw, const void* w13, const fmoe_scales* sc, char* W,
                        cudaStream_t s) {
-  int32_t* ids = reinterpret_cast<int32_t*>(W + L.ids);
-  float* tw = reinterpret_cast<float*>(W + L.tw);
-  int32_t* counts = reinterpret_cast<int32_t*>(W + L.counts);
-  int32_t* offsets = reinterpret_cast<int32_t*>(W + L.offsets);
-  int32_t* rows = reinterpret_cast<int32_t*>(W + L.rows);
-  int32_t* inv = reinterpret_cast<int32_t*>(W + L.inv);
-  float* y = reinterpret_cast<float*>(W + L.y);
   bool plan_two_back = true;  // the plan-writing launch is followed by the gather launch
   if (fuse_route_permute(L)) {
-    const PermuteArgs p = permute_args(d, L, ids, sc, counts, offsets, rows, inv, W, true);
-    const GatherArgs g = gather_args(d, L, x, rows, W + L.a_perm, W);
+    const PermuteArgs p = permute_args(d, L, b.ids, sc, b.counts, b.offsets, b.rows, b.inv, W, true);
+    const GatherArgs g = gather_args(d, L, x, b.rows, W + L.a_perm, W);
     const bool fg = fuse_route_gather(d, L);
-    FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s, &p, fg ? &g : nullptr));
+    FMOE_TRY(route_impl(d, L, x, rw, b.ids, b.tw, W, s, &p, fg ? &g : nullptr));
     if (!fg) FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
     plan_two_back = !fg;
   } else {
-    FMOE_TRY(route_impl(d, L, x, rw, ids, tw, W, s));
-    FMOE_TRY(permute_impl(d, L, ids, x, sc, counts, offsets, rows, inv, W + L.a_perm, W, s,
-                          /*with_plan=*/true));
+    FMOE_TRY(route_impl(d, L, x, rw, b.ids, b.tw, W, s));
+    FMOE_TRY(permute_impl(d, L, b.ids, x, sc, b.counts, b.offsets, b.rows, b.inv, W + L.a_perm, W,
+                          s, /*with_plan=*/true));
   }
-  FMOE_TRY(experts_impl(d, L, W + L.a_perm, offsets, rows, tw, w13, w2, sc, y, W, s,
-                        /*plan_done=*/true, /*fused_out=*/out, ids, inv, plan_two_back));
+  return experts_first(d, L, W + L.a_perm, b.offsets, b.rows, b.tw, w13, sc, W, s,
+                       /*plan_done=*/true, plan_two_back);
+}
+
+// Step a4 and a5 of the one-call path: bf16 `out`, or (a tensor-parallel shard) the fp32
+// sums `out_f32` with the max |h| taken from amax_in.
+fmoe_status second_half(const fmoe_dims& d, const Layout& L, const OneCall& b, const void* w2,
+                        const fmoe_scales* sc, void* out, float* out_f32, const float* amax_in,
+                        char* W, cudaStream_t s) {
+  FMOE_TRY(experts_second(d, L, b.offsets, b.rows, b.tw, w2, sc, b.y, W, s, out, out_f32, b.ids,
+                          b.inv, amax_in));
   if (L.swap) return FMOE_OK;  // combined by combine_partials
-  return combine_impl(d, y, inv, out, s);
+  return combine_impl(d, b.y, b.inv, out, s, out_f32);
+}
+
+fmoe_status fused_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
+                       const void* w13, const void* w2, const fmoe_scales* sc, void* out, char* W,
+                       cudaStream_t s) {
+  const OneCall b(L, W);
+  FMOE_TRY(first_half(d, L, b, x, rw, w13, sc, W, s));
+  return second_half(d, L, b, w2, sc, out, nullptr, nullptr, W, s);
 }
 
 }  // namespace
@@ -659,6 +726,58 @@ fmoe_status fused_moe(const fmoe_dims* dims, const void* x, const void* router_w
   FMOE_TRY(check_ws(L, ws, ws_bytes));
   return fused_impl(*dims, L, x, router_w, w13, w2, scales, out, static_cast<char*>(ws),
                     static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_tp_begin(const fmoe_dims* dims, const void* x, const void* router_w,
+                               const void* w13, const fmoe_scales* scales, float* amax_h,
+                               void* ws, size_t ws_bytes, fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(x, router_w, w13));
+  if (amax_h == nullptr) return FMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(amax_h) & 3u) != 0) return FMOE_ERR_UNSUPPORTED;
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  char* W = static_cast<char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const OneCall b(L, W);
+  FMOE_TRY(first_half(*dims, L, b, x, router_w, w13, scales, W, s));
+  AmaxReduceArgs r{};
+  r.amax_part = reinterpret_cast<const float*>(W + L.amax_h);
+  r.hdr = reinterpret_cast<const WsHeader*>(W + L.hdr);
+  r.amax_out = amax_h;
+  r.fp8 = L.fp8 ? 1 : 0;
+  FMOE_LAUNCH("amax_reduce", launch_amax_reduce(r, s), s);
+  return FMOE_OK;
+}
+
+fmoe_status fused_moe_tp_end(const fmoe_dims* dims, const void* w2, const fmoe_scales* scales,
+                             const float* amax_h, float* out_partial, void* ws, size_t ws_bytes,
+                             fmoe_stream stream) {
+  FMOE_TRY(check_dims(dims));
+  if (dims->T == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(w2, out_partial));
+  if (amax_h == nullptr) return FMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(amax_h) & 3u) != 0) return FMOE_ERR_UNSUPPORTED;
+  FMOE_TRY(check_fp8_scales(*dims, scales));
+  if (dims->wdtype == FMOE_FP8_E4M3) FMOE_TRY(check_ptrs(scales->w13_scale, scales->w2_scale));
+  const Layout L = make_layout(*dims);
+  FMOE_TRY(check_ws(L, ws, ws_bytes));
+  char* W = static_cast<char*>(ws);
+  const OneCall b(L, W);
+  return second_half(*dims, L, b, w2, scales, nullptr, out_partial, amax_h, W,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fused_moe_tp_finish(int64_t n, const float* out_sum, void* out, fmoe_stream stream) {
+  if (n < 0) return FMOE_ERR_INVALID_ARG;
+  if (n == 0) return FMOE_OK;
+  FMOE_TRY(check_ptrs(out_sum, out));
+  if (n % 8 != 0 || n >= (int64_t(1) << 40)) return FMOE_ERR_UNSUPPORTED;
+  return cuda_status(launch_to_bf16(out_sum, static_cast<uint16_t*>(out), static_cast<size_t>(n),
+                                    num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 fmoe_status fused_moe_host_io(const fmoe_dims* dims, const void* x_host, const void* router_w,

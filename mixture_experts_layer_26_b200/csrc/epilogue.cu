@@ -10,7 +10,10 @@
 //   the routing weight of the row.
 // combine: out[t] = bf16( sum over j < k of y[inv_perm[t*k+j]] ), fp32 adds in j order
 //   ("expert aggregation", codebridge-ai.com blog on the AWS MoE kernels,
-//   "2. Backend routing: Triton over CUTLASS").
+//   "2. Backend routing: Triton over CUTLASS"); one shard of a tensor-parallel layer
+//   writes the fp32 sums instead, and to_bf16 rounds the sum over the shards.
+// amax_reduce (tensor parallelism): this shard's max |h| as one device word, for the
+//   cross-shard max that fixes the per-tensor scale of h.
 //
 // All four are HBM/L2-bound and use 16-byte vector accesses; their grids are a
 // multiple of the SM count.
@@ -112,8 +115,12 @@ __global__ void __launch_bounds__(kEwThreads) quant_h_kernel(QuantHArgs a) {
   griddep_launch_dependents();
   if (threadIdx.x < 32) {
     float m = 0.f;
-    const int n = a.hdr->amax_h_count;
-    for (int i = threadIdx.x; i < n; i += 32) m = fmaxf(m, a.amax_part[i]);
+    if (a.amax_in != nullptr) {
+      m = *a.amax_in;  // the max over every shard of a tensor-parallel layer
+    } else {
+      const int n = a.hdr->amax_h_count;
+      for (int i = threadIdx.x; i < n; i += 32) m = fmaxf(m, a.amax_part[i]);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (threadIdx.x == 0) {
@@ -210,6 +217,17 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* acc) {
   return o;
 }
 
+// One combined output row segment of 8 values: bf16 (round to nearest even), or the fp32
+// sums themselves when the layer is one shard of a tensor-parallel group.
+__device__ __forceinline__ void store_out(uint16_t* out, float* out_f32, size_t o, const float* acc) {
+  if (out_f32 != nullptr) {
+    reinterpret_cast<float4*>(out_f32 + o)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    reinterpret_cast<float4*>(out_f32 + o)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  } else {
+    *reinterpret_cast<uint4*>(out + o) = pack_bf16x8(acc);
+  }
+}
+
 // Same arithmetic, in the same order, as finalize2 followed by combine.
 __global__ void __launch_bounds__(kEwThreads) combine_partials_kernel(CombinePartialsArgs a) {
   griddep_wait();
@@ -246,7 +264,7 @@ __global__ void __launch_bounds__(kEwThreads) combine_partials_kernel(CombinePar
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = (j == 0) ? y[i] : acc[i] + y[i];
     }
-    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = pack_bf16x8(acc);
+    store_out(a.out, a.out_f32, static_cast<size_t>(t) * a.H + c, acc);
   }
 }
 
@@ -272,7 +290,35 @@ __global__ void __launch_bounds__(kEwThreads) combine_kernel(CombineArgs a) {
         acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
       }
     }
-    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.H + c) = pack_bf16x8(acc);
+    store_out(a.out, a.out_f32, static_cast<size_t>(t) * a.H + c, acc);
+  }
+}
+
+// Tensor parallelism: the largest of this shard's per-CTA max |h| partials.
+__global__ void amax_reduce_kernel(AmaxReduceArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  float m = 0.f;
+  if (a.fp8) {
+    const int n = a.hdr->amax_h_count;
+    for (int i = threadIdx.x; i < n; i += 32) m = fmaxf(m, a.amax_part[i]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (threadIdx.x == 0) *a.amax_out = m;
+}
+
+// Tensor parallelism: bf16 rounding of the summed partial outputs, 8 values per thread.
+__global__ void __launch_bounds__(kEwThreads) to_bf16_kernel(const float* in, uint16_t* out,
+                                                             size_t n8) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (size_t v = blockIdx.x * static_cast<size_t>(kEwThreads) + threadIdx.x; v < n8;
+       v += static_cast<size_t>(gridDim.x) * kEwThreads) {
+    const float4 a0 = reinterpret_cast<const float4*>(in)[2 * v];
+    const float4 a1 = reinterpret_cast<const float4*>(in)[2 * v + 1];
+    const float acc[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    reinterpret_cast<uint4*>(out)[v] = pack_bf16x8(acc);
   }
 }
 
@@ -328,6 +374,15 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
 cudaError_t launch_wait_selftest(WsHeader* hdr, uint64_t budget_ns, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>(hdr, budget_ns);
   return cudaGetLastError();
+}
+
+cudaError_t launch_amax_reduce(const AmaxReduceArgs& a, cudaStream_t s) {
+  return launch_k(amax_reduce_kernel, dim3(1), dim3(32), 0, s, a);
+}
+
+cudaError_t launch_to_bf16(const float* in, uint16_t* out, size_t n, int num_sms, cudaStream_t s) {
+  const size_t n8 = n / 8;
+  return launch_k(to_bf16_kernel, dim3(ew_grid(n8, num_sms)), dim3(kEwThreads), 0, s, in, out, n8);
 }
 
 cudaError_t launch_combine_partials(const CombinePartialsArgs& a, int num_sms, cudaStream_t s) {

@@ -178,11 +178,27 @@ struct QuantHArgs {
   const uint16_t* h_bf16;   // [R, I] bf16 (when non-null)
   uint8_t* hq;              // [R, I] e4m3
   const float* amax_part;
+  const float* amax_in;     // non-null: max |h| taken from this device word (tensor
+                            // parallelism: the max over every shard) instead of amax_part
   WsHeader* hdr;
   int R, I;
   float a2_static;
 };
 cudaError_t launch_quant_h(const QuantHArgs& a, int num_sms, cudaStream_t s);
+
+// Tensor parallelism: reduce this shard's per-CTA max |h| partials into one device word
+// (0 in the bf16 format, which has no second quantisation).
+struct AmaxReduceArgs {
+  const float* amax_part;
+  const WsHeader* hdr;      // amax_h_count
+  float* amax_out;
+  int fp8;
+};
+cudaError_t launch_amax_reduce(const AmaxReduceArgs& a, cudaStream_t s);
+
+// Tensor parallelism: out = bf16(sum) of the shards' summed fp32 partial outputs, round to
+// nearest even; n a multiple of 8.
+cudaError_t launch_to_bf16(const float* in, uint16_t* out, size_t n, int num_sms, cudaStream_t s);
 
 struct Finalize2Args {
   const float* part;        // [S][R][H]
@@ -207,7 +223,8 @@ struct CombinePartialsArgs {
   const float* topk_w;      // [R]
   const float* w2_scale;    // [E] or null
   const WsHeader* hdr;
-  uint16_t* out;            // [T, H] bf16
+  uint16_t* out;            // [T, H] bf16, or
+  float* out_f32;           // [T, H] fp32 sums before rounding (when non-null)
   int T, H, k, E;
   int fp8;
 };
@@ -219,7 +236,8 @@ cudaError_t launch_wait_selftest(WsHeader* hdr, uint64_t budget_ns, cudaStream_t
 struct CombineArgs {
   const float* y;           // [R, H]
   const int32_t* inv_perm;  // [R]
-  uint16_t* out;            // [T, H] bf16
+  uint16_t* out;            // [T, H] bf16, or
+  float* out_f32;           // [T, H] fp32 sums before rounding (when non-null)
   int T, H, k;
 };
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);

@@ -317,14 +317,21 @@ def silu(g: np.ndarray) -> np.ndarray:
 
 
 def experts(a_perm, offsets, sorted_rows, topk_w, w13, w2, H, I, E,
-            fp8=True, s1=np.float32(1), w13_scale=None, w2_scale=None, a2_scale=0.0):
+            fp8=True, s1=np.float32(1), w13_scale=None, w2_scale=None, a2_scale=0.0,
+            amax2=None):
     """Per-expert gated MLP on the permuted rows.
 
     Returns y [R,H] float64 (already multiplied by the routing weight of its
     row), h [R,I] float32, hq (codes or bf16 bits) [R,I], s2.
     FP8: g,u = (Aq_e . W1_e^T, Aq_e . W3_e^T) * (s1*sw13[e]) in fp64; h = SiLU(g)*u
     stored as fp32; hq = e4m3(h * inv2) with the global amax of h (R4);
-    Y = (hq_e . W2_e^T) * (s2*sw2[e]).  bf16 (R7): no scales; h -> bf16."""
+    Y = (hq_e . W2_e^T) * (s2*sw2[e]).  bf16 (R7): no scales; h -> bf16.
+
+    amax2: the max |h| the per-tensor scale of h is taken from; None means the max of
+    this call's h.  One shard of the layer split over the intermediate features (the
+    tensor parallelism the pages measure at 8 ways: agentic-affairs.com, third change)
+    holds a slice of h; given the max over the whole layer's h, its codes are the
+    unsharded layer's codes for those features (R4 takes the scale over all of h)."""
     R = a_perm.shape[0]
     A = e4m3_decode(a_perm) if fp8 else bf16_to_f32(a_perm).astype(np.float64)
     h = np.zeros((R, I), dtype=np.float32)
@@ -338,8 +345,9 @@ def experts(a_perm, offsets, sorted_rows, topk_w, w13, w2, H, I, E,
         g, u = acc[:, :I] * sc, acc[:, I:] * sc                 # R6
         h[r0:r1] = (silu(g) * u).astype(np.float32)
     if fp8:
-        amax2 = np.float32(np.abs(h).max()) if h.size else np.float32(0)
-        s2, inv2 = act_scales(amax2, a2_scale)
+        if amax2 is None:
+            amax2 = np.float32(np.abs(h).max()) if h.size else np.float32(0)
+        s2, inv2 = act_scales(np.float32(amax2), a2_scale)
         hq = quantize(h, inv2)
         B = e4m3_decode(hq)
     else:

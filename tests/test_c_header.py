@@ -42,7 +42,7 @@ def test_header_is_c99_and_host_calls_work(tmp_path):
                     f"-Wl,-rpath,{LIBDIR}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
     abi, ws_ok, launches, bad_ws, rope = (int(v) for v in out[0].split())
-    assert abi == 3 and ws_ok == 1 and bad_ws == 0
+    assert abi == 4 and ws_ok == 1 and bad_ws == 0
     # router (+ permutation and plan: 144 rows), gather (144 x 7168 x 2 B > 128 KB), gemm1,
     # finalize1, quant_h, gemm2, combine of the split-K partials
     assert launches == 7

@@ -23,7 +23,7 @@ def header_symbols():
 
 def test_header_symbols_are_exported():
     syms = header_symbols()
-    assert len(syms) == 17
+    assert len(syms) == 20
     assert set(syms) == set(capi.EXPORTED)
     lib = ctypes.CDLL(capi.LIB_PATH)
     for s in syms:
@@ -31,7 +31,7 @@ def test_header_symbols_are_exported():
 
 
 def test_abi_version_and_strings():
-    assert capi.abi_version() == 3
+    assert capi.abi_version() == 4
     for code, name in [(0, "FMOE_OK"), (1, "FMOE_ERR_INVALID_ARG"), (2, "FMOE_ERR_UNSUPPORTED"),
                        (3, "FMOE_ERR_WORKSPACE"), (4, "FMOE_ERR_CUDA"), (5, "FMOE_ERR_TIMEOUT"),
                        (6, "FMOE_ERR_DEVICE_BOUNDS")]:

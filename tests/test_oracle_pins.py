@@ -522,3 +522,56 @@ def test_shared_expert_adds_a_dense_gated_mlp():
     h = h.to(torch.bfloat16).to(torch.float64)                      # R7: h rounded to bf16
     y = (h @ w2.T).numpy()
     assert np.abs(diff - y).max() <= 1e-9 * np.abs(y).max()
+
+
+# ----------------------------------------------------------------------------- sharding
+
+def _shard(w13, w2, r, n):
+    """Plain numpy slices of shard r of n over the intermediate features (independent of
+    the package's torch helper)."""
+    I = w2.shape[2]
+    m = I // n
+    cols = np.arange(r * m, (r + 1) * m)
+    return np.concatenate([w13[:, cols], w13[:, I + cols]], axis=1), w2[:, :, cols], cols
+
+
+@pytest.mark.parametrize("n", [2, 4])
+@pytest.mark.parametrize("wdtype", ["fp8", "bf16"])
+def test_sharded_expert_networks_reassemble_the_layer(n, wdtype):
+    """Splitting the intermediate features over n shards, each given the max |h| of the
+    whole layer (amax2), reproduces the unsharded layer: every shard's h and its codes
+    are the unsharded columns bit for bit, and the shards' outputs add up to the
+    unsharded output (the contraction over I splits into a sum over shards)."""
+    T, H, I, E, k = 9, 256, 512, 4, 2
+    s = tiny_shape(T, H, I, E, k, wdtype)
+    inp = minp.make_inputs(s, seed=21)
+    d = np_inputs(inp)
+    fp8 = d["fp8"]
+    full = run_oracle(O, inp)
+    ids, w = full["topk_ids"], full["topk_w"]
+    a_perm, s1 = full["a_perm"], full["s1"]
+    amax_full = np.float32(np.abs(full["h"]).max())
+    y_sum = np.zeros_like(full["y"])
+    local_codes_differ = False
+    for r in range(n):
+        w13_r, w2_r, cols = _shard(d["w13"], d["w2"], r, n)
+        y_r, h_r, hq_r, s2_r = O.experts(a_perm, full["offsets"], full["sorted_rows"], w, w13_r,
+                                         w2_r, H, I // n, E, fp8, s1, d["w13_scale"],
+                                         d["w2_scale"], amax2=amax_full if fp8 else None)
+        assert np.array_equal(h_r, full["h"][:, cols])
+        assert np.array_equal(hq_r, full["hq"][:, cols])
+        assert s2_r == full["s2"]
+        y_sum += y_r
+        if fp8:   # a shard scaled by its own max would quantise differently
+            _, _, hq_own, _ = O.experts(a_perm, full["offsets"], full["sorted_rows"], w, w13_r,
+                                        w2_r, H, I // n, E, fp8, s1, d["w13_scale"],
+                                        d["w2_scale"])
+            local_codes_differ |= not np.array_equal(hq_own, hq_r)
+    assert np.abs(y_sum - full["y"]).max() <= 1e-12 * np.abs(full["y"]).max()
+    if fp8:
+        assert local_codes_differ
+    # amax2 equal to the call's own max is the default
+    y_a, _, hq_a, _ = O.experts(a_perm, full["offsets"], full["sorted_rows"], w, d["w13"], d["w2"],
+                                H, I, E, fp8, s1, d["w13_scale"], d["w2_scale"],
+                                amax2=amax_full if fp8 else None)
+    assert np.array_equal(hq_a, full["hq"]) and np.array_equal(y_a, full["y"])
