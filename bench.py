@@ -718,6 +718,46 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_route_only(args, rank, world, local_rank):
+    """`--step route`: the routing step alone (fused_moe_route: the router kernel and its
+    tail) on the workload's x and router_w, back to back; no expert weights are allocated,
+    so the run is small enough for a detailed profile of the router.  Prints one line with
+    the mean time per call."""
+    from mixture_experts_layer_26_b200 import capi
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = minp.shape(args.workload, args.T)
+    x, wr = minp.make_activations(s, seed=0)
+    bias = minp.make_router_bias(s, seed=0)
+    routing = None
+    if s.grouped is not None:
+        routing = capi.make_routing(*s.grouped, bias.to(dev), n_shared=s.n_shared)
+    elif s.n_shared:
+        routing = capi.make_softmax_routing(s.n_shared)
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, s.wdtype == "fp8", routing=routing)
+    ws = capi.alloc_workspace(dims, dev)
+    ids = torch.empty(s.R, dtype=torch.int32, device=dev)
+    tw = torch.empty(s.R, dtype=torch.float32, device=dev)
+    xd, wd = x.to(dev), wr.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        capi.fused_moe_route(dims, xd, wd, ids, tw, ws, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        capi.fused_moe_route(dims, xd, wd, ids, tw, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert capi.fused_moe_get_device_status(ws, stream) == capi.FMOE_OK
+    us = 1e3 * e0.elapsed_time(e1) / args.steps
+    if rank == 0:
+        print(json.dumps({"step": "route", "workload": workload_config(s)["workload"],
+                          "us_per_call": round(us, 2), "calls": args.steps,
+                          "fmas": s.T * s.E * s.H, "tokens_per_s": round(s.T / (us / 1e6), 1)}))
+    return 0
+
+
 def run_tp_ours(args, rank, world, local_rank):
     """Tensor parallelism over the intermediate features: rank r of N holds shard r of
     every expert and the N ranks compute ONE batch together (strong scaling).  A step is
@@ -1010,6 +1050,8 @@ def main(argv=None):
                     help="tokens (default: the workload's largest; 4096 for the default workload)")
     ap.add_argument("--variant", default="auto", choices=["auto", "swap_ab", "normal", "normal_pair"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--step", choices=["layer", "route"], default="layer",
+                    help="route: time the routing step alone (no expert weights allocated)")
     ap.add_argument("--tp", action="store_true",
                     help="tensor parallelism: the ranks share one layer, each holding I/N")
     ap.add_argument("--no-extras", action="store_true",
@@ -1030,6 +1072,8 @@ def main(argv=None):
         return run_rope_ours(args, rank, world, local_rank)
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.step == "route":
+        return run_route_only(args, rank, world, local_rank)
     if args.tp:
         return run_tp_ours(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)

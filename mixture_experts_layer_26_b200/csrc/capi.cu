@@ -29,7 +29,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   bool fp8 = false, swap = false, pair = false;
   int R = 0, chunk_rows = 0, max_chunks = 0, s1max = 0, s2max = 0;
-  size_t hdr = 0, counters = 0, amax_x = 0, amax_h = 0, chunks = 0, logits = 0;
+  size_t hdr = 0, counters = 0, amax_x = 0, amax_h = 0, chunks = 0, logits = 0, ready = 0;
   size_t ids = 0, tw = 0, counts = 0, offsets = 0, rows = 0, inv = 0;
   size_t x_in = 0, out_dev = 0, a_perm = 0, p1 = 0, h = 0, hq = 0, p2 = 0, y = 0;
   size_t total = 0;
@@ -110,6 +110,7 @@ Layout make_layout(const fmoe_dims& d) {
   L.logits = take(static_cast<size_t>(T) * E * 4);
   L.amax_h = take(static_cast<size_t>(kAmaxSlots) * 4);
   L.chunks = take(static_cast<size_t>(L.max_chunks) * sizeof(Chunk));
+  L.ready = take(static_cast<size_t>(L.max_chunks) * 4);
   L.ids = take(static_cast<size_t>(R) * 4);
   L.tw = take(static_cast<size_t>(R) * 4);
   L.counts = take(static_cast<size_t>(E) * 4);
@@ -199,6 +200,22 @@ bool encode_map(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint
   return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 rows [rows, inner] without swizzle, boxes of 256 columns x box_rows rows (the
+// tiled router's x and router_w slices); rows past the end read as zeros.
+bool encode_rows_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                     uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tma_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {256u, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline fmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA; }
 
 #define FMOE_TRY(expr)                   \
@@ -263,8 +280,13 @@ PlanParams plan_params(const fmoe_dims& d, const Layout& L, char* W) {
   p.s1max = std::max(L.s1max, 1);
   p.s2max = std::max(L.s2max, 1);
   p.num_sms = num_sms();
+  p.ready = reinterpret_cast<int32_t*>(W + L.ready);
   return p;
 }
+
+// The CTA-pair FP8 second contraction quantises h itself (no quant_h launch) unless the
+// max |h| comes from outside the call (a tensor-parallel shard).
+bool fuse_quant_h(const Layout& L, const float* amax_in) { return L.pair && L.fp8 && amax_in == nullptr; }
 
 // Small batches whose routed rows fit one CTA's permutation: the router's final CTA
 // also runs permute (+ plan) and, when the gathered rows are at most 128 KB, the gather.
@@ -315,9 +337,20 @@ fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const
       a.gather = *fused_gather;
     }
   }
-  FMOE_LAUNCH(fused_perm == nullptr ? "router"
-                                    : (fused_gather == nullptr ? "router_permute" : "router_permute_gather"),
-              launch_router(a, s), s);
+  const char* name = fused_perm == nullptr ? "router"
+                                            : (fused_gather == nullptr ? "router_permute"
+                                                                       : "router_permute_gather");
+  if (router_use_tiled(d.T, d.E, a.num_sms)) {
+    RouterMaps m;
+    if (!encode_rows_map(&m.x, x, static_cast<uint64_t>(d.H), static_cast<uint64_t>(d.T),
+                         static_cast<uint32_t>(router_tile_tokens(d.E))) ||
+        !encode_rows_map(&m.wr, rw, static_cast<uint64_t>(d.H), static_cast<uint64_t>(d.E),
+                         static_cast<uint32_t>(router_tile_experts(d.E))))
+      return FMOE_ERR_CUDA;
+    FMOE_LAUNCH(name, launch_router_tiled(a, m, s), s);
+  } else {
+    FMOE_LAUNCH(name, launch_router(a, s), s);
+  }
   return FMOE_OK;
 }
 
@@ -471,7 +504,8 @@ fmoe_status experts_second(const fmoe_dims& d, const Layout& L, const int32_t* o
   float* hbuf = reinterpret_cast<float*>(W + L.h);
   void* hq = W + L.hq;
 
-  if (fp8) {
+  const bool fq = fuse_quant_h(L, amax_in);
+  if (fp8 && !fq) {
     QuantHArgs q{};
     q.h = hbuf;
     q.h_bf16 = nullptr;
@@ -498,6 +532,13 @@ fmoe_status experts_second(const fmoe_dims& d, const Layout& L, const int32_t* o
   g2.Nout = H;
   g2.rows_per_expert = H;
   g2.prefetch_w = 1;  // the chunk list was written at least two launches back (gemm1 between)
+  if (fq) {
+    g2.fuse_quant = 1;
+    g2.q_h = hbuf;
+    g2.q_hq = static_cast<uint8_t*>(hq);
+    g2.q_ready = reinterpret_cast<int32_t*>(W + L.ready);
+    g2.q_a2_static = sc != nullptr ? sc->a2_scale : 0.f;
+  }
   if (L.pair)
     FMOE_LAUNCH("gemm2_pair", launch_gemm_pair(g2, fp8, 2, sms, s), s);
   else
@@ -804,8 +845,9 @@ int32_t fused_moe_launches_per_call(const fmoe_dims* dims) {
   if (check_dims(dims) != FMOE_OK) return -1;
   if (dims->T == 0) return 0;
   const Layout L = make_layout(*dims);
-  // router [+ permute (+plan) [+ gather]], gemm1, [finalize1], [quant_h], gemm2, combine
-  int n = 4 + (L.fp8 ? 1 : 0) + (L.swap ? 1 : 0);
+  // router [+ permute (+plan) [+ gather]], gemm1, [finalize1], [quant_h], gemm2, combine;
+  // the CTA-pair FP8 second contraction quantises h itself
+  int n = 4 + (L.fp8 && !fuse_quant_h(L, nullptr) ? 1 : 0) + (L.swap ? 1 : 0);
   if (!fuse_route_permute(L)) n += 2;        // permute, gather
   else if (!fuse_route_gather(*dims, L)) n += 1;  // gather
   return n;

@@ -60,6 +60,7 @@ struct PlanParams {
   int kblocks1, kblocks2;  // K blocks of each contraction
   int s1max, s2max;        // largest split-K factors the workspace holds
   int num_sms;
+  int32_t* ready;          // [max_chunks] per-chunk counters zeroed with the plan, or null
 };
 
 struct PermuteArgs {
@@ -117,6 +118,19 @@ struct RouterArgs {
 // Token tiles that may split their experts over several CTAs (counters in the header area).
 constexpr int kRouterMaxTiles = 4096;
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+
+// Tiled router for large T*E (router.cu): TMA tensor maps of x [T, H] and router_w [E, H],
+// bf16 without swizzle, boxes of 256 columns x router_tile_tokens(E) token rows and
+// x router_tile_experts(E) expert rows.
+struct alignas(64) RouterMaps {
+  CUtensorMap x;
+  CUtensorMap wr;
+};
+int router_tile_tokens(int E);
+int router_tile_experts(int E);
+// Whether (T, E) has enough token x expert tiles for the tiled router to fill the GPU.
+bool router_use_tiled(int T, int E, int num_sms);
+cudaError_t launch_router_tiled(const RouterArgs& a, const RouterMaps& m, cudaStream_t s);
 int router_tokens_per_cta(int T, int H, int E, int num_sms);
 int router_experts_per_warp(int E);
 
@@ -151,6 +165,14 @@ struct GemmArgs {
   int prefetch_w;          // 1: the chunk list was written at least two launches earlier,
                            // so weight tiles may be loaded before griddepcontrol.wait
   uint64_t wait_budget_ns;
+  // CTA-pair second contraction, FP8: quantise h inside the kernel (launch_gemm_pair with
+  // fuse_quant = 1) instead of a separate quant_h pass -- see gemm_pair.cu
+  int fuse_quant;
+  const float* q_h;        // [R, I] fp32 h
+  uint8_t* q_hq;           // [R, I] e4m3 out: the activations map_x reads
+  int32_t* q_ready;        // [max_chunks] CTAs that finished their share of each chunk (zero
+                           // at launch: the plan zeroes them)
+  float q_a2_static;       // > 0: static scale of h
 };
 // gemm = 1 (w13, gate/up) or 2 (w2); fp8 selects kind::f8f6f4 vs kind::f16.
 cudaError_t launch_gemm(const GemmArgs& a, bool fp8, bool swap_ab, int gemm, int num_sms,

@@ -24,6 +24,7 @@
 // a timeout the pair reconciles the copies either CTA issued, waits (bounded) for them
 // and for the MMAs in flight, frees its TMEM and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "fmoe_kernels.h"
 
@@ -161,9 +162,58 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_ma
 }
 
 // ------------------------------------------------------------------------------------
+// in-kernel quantisation of h (second contraction, FP8)
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Generic-proxy global writes before, async-proxy (TMA) reads after.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void quant_warps_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t e4m3x4_q(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// The per-tensor scale of h from the first contraction's per-CTA max |h| partials (one
+// warp; every warp that calls it gets the same values): s2 = amax/448 and 448/amax, each one
+// fp32 division, 1 for amax = 0, or a static scale s and 1/s -- the quant_h pass's rule.
+__device__ __forceinline__ void h_scales(const GemmArgs& a, float& amax, float& s2, float& inv2) {
+  const int lane = threadIdx.x & 31;
+  const int n = a.hdr->amax_h_count;
+  float m = 0.f;
+  for (int i = lane; i < n; i += 32) m = fmaxf(m, a.amax_part[i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  amax = m;
+  s2 = 1.f;
+  inv2 = 1.f;
+  if (a.q_a2_static > 0.f) {
+    s2 = a.q_a2_static;
+    inv2 = 1.0f / a.q_a2_static;
+  } else if (m > 0.f) {
+    s2 = m / 448.0f;
+    inv2 = 448.0f / m;
+  }
+}
+
+// ------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;       // producer, MMA, 4 epilogue warps
+constexpr int kQuantThreads = 320;  // + 4 warps quantising h (second contraction, FP8)
 constexpr int kTile = 128 * 128;        // bytes of a 128-row x 128-byte operand tile
 constexpr int kStageBytes = 2 * kTile;  // per CTA and K step: 128 token rows + 128 weight rows
 constexpr int kStages = 7;
@@ -187,7 +237,7 @@ struct PairCtl {
 };
 
 struct PairUnit {
-  int e, row0, nrows, tile, nch;
+  int e, row0, nrows, tile, nch, chunk;
 };
 
 __device__ __forceinline__ uint64_t policy_evict_normal() {
@@ -203,8 +253,10 @@ __device__ __forceinline__ PairUnit decode_pair_unit(long u, const Chunk* chunks
   const int q = static_cast<int>(u / tiles);
   const Chunk cq = chunks[q];
   const long local = u - static_cast<long>(cq.cb) * tiles;
-  const Chunk cc = chunks[cq.cb + static_cast<int>(local % cq.nch)];
+  const int ci = cq.cb + static_cast<int>(local % cq.nch);
+  const Chunk cc = chunks[ci];
   PairUnit t;
+  t.chunk = ci;
   t.tile = static_cast<int>(local / cq.nch);
   t.e = cc.e;
   t.row0 = cc.row0;
@@ -213,8 +265,10 @@ __device__ __forceinline__ PairUnit decode_pair_unit(long u, const Chunk* chunks
   return t;
 }
 
-template <bool kFp8, int kGemm>
-__global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+template <bool kFp8, int kGemm, bool kQuant>
+__global__ void __launch_bounds__(kQuant ? kQuantThreads : kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmArgs a) {
+  static_assert(!kQuant || (kFp8 && kGemm == 2), "h is quantised in the FP8 second contraction");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ PairCtl ctl;
 
@@ -293,7 +347,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
         tma_load_2d_pair(smem + st * kStageBytes + kTile, &a.map_w, leader_full(st), kb * kBK, wrow,
                          t.nch > 1 ? pol_w_shared : pol_w_once);
       };
+      // kQuant: the token rows of a chunk are e4m3 codes the quantiser warps of every CTA
+      // write; wait (bounded) until all CTAs have counted the chunk done.  A wait that runs
+      // out raises the abort flag; the load is still issued so that both CTAs of the pair
+      // issue the same fills and the teardown below stays exact.
+      int ready_upto = 0;
+      auto wait_ready = [&](int c) {
+        if constexpr (kQuant) {
+          if (c < ready_upto || *abort_flag) return;
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(a.q_ready + c) < static_cast<int>(gridDim.x)) {
+            if (*abort_flag) return;
+            if (globaltimer_ns() - t0 > budget) {
+              *abort_flag = 1;
+              record_status(a.status, ST_TIMEOUT);
+              return;
+            }
+            __nanosleep(100);
+          }
+          ready_upto = c + 1;
+          fence_proxy_async_global();
+        }
+      };
       auto load_x = [&](int st, const PairUnit& t, int kb) {
+        wait_ready(t.chunk);
         tma_load_2d_pair(smem + st * kStageBytes, &a.map_x, leader_full(st), kb * kBK,
                          t.row0 + 128 * static_cast<int>(rank), pol_x);
       };
@@ -421,9 +498,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
         mbar_wait(&ctl.drain, 0, &dummy, a.status, budget);
       }
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------- epilogue
     if (prefetch) griddep_wait();  // scales and routing weights of this call
+    float s2_local = 1.f;
+    if constexpr (kQuant) {
+      float amax_unused, inv_unused;
+      h_scales(a, amax_unused, s2_local, inv_unused);
+    }
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
     const int r = static_cast<int>(rank) * 128 + q * 32 + lane;  // row within the unit
     int acc = 0;
@@ -474,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
         }
       } else {
         // lane = token row0 + r; columns = output features tile*256 ..
-        const float sc = kFp8 ? a.hdr->s2 * a.w_scale[t.e] : 1.f;
+        const float sc = kFp8 ? (kQuant ? s2_local : a.hdr->s2) * a.w_scale[t.e] : 1.f;
         const int src_row = valid ? a.sorted_rows[t.row0 + r] : 0;
         const bool in_range = src_row >= 0 && src_row < a.R;
         if (valid && !in_range) record_status(a.status, ST_BOUNDS);
@@ -505,6 +587,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       if (lane == 0) atomicMax(&ctl.amax_bits, __float_as_int(amax));
+    }
+  } else {
+    // ------------------------------------------------------------- quantisation of h
+    // Every CTA quantises an equal share of every chunk, chunks in the order of the chunk
+    // list (the order the units need them), and counts the chunk done; the producers of all
+    // CTAs load a chunk's token rows once every CTA has counted it.
+    if constexpr (kQuant) {
+      griddep_wait();  // h and the max |h| partials of the first contraction are complete
+      float amax2, s2, inv2;
+      h_scales(a, amax2, s2, inv2);
+      WsHeader* hw = a.hdr_w;
+      if (blockIdx.x == 0 && threadIdx.x == 6 * 32) {  // recorded for the debug scalars
+        hw->amax_h = amax2;
+        hw->s2 = s2;
+        hw->inv2 = inv2;
+      }
+      const int qt = threadIdx.x - 6 * 32;  // 0..127
+      const int nc = ctl.n_chunks;
+      const size_t G = gridDim.x;
+      for (int c = 0; c < nc; ++c) {
+        const Chunk ch = a.chunks[c];
+        const size_t base = static_cast<size_t>(ch.row0) * a.I;  // elements
+        const size_t n16 = static_cast<size_t>(ch.nrows) * (a.I / 16);
+        const size_t per = (n16 + G - 1) / G;
+        const size_t v0 = min(n16, blockIdx.x * per), v1 = min(n16, v0 + per);
+        const float4* src = reinterpret_cast<const float4*>(a.q_h + base);
+        uint4* dst = reinterpret_cast<uint4*>(a.q_hq + base);
+        for (size_t v = v0 + qt; v < v1; v += 128) {
+          const float4 f0 = __ldcs(src + 4 * v), f1 = __ldcs(src + 4 * v + 1);
+          const float4 f2 = __ldcs(src + 4 * v + 2), f3 = __ldcs(src + 4 * v + 3);
+          uint4 q;
+          q.x = e4m3x4_q(f0.x * inv2, f0.y * inv2, f0.z * inv2, f0.w * inv2);
+          q.y = e4m3x4_q(f1.x * inv2, f1.y * inv2, f1.z * inv2, f1.w * inv2);
+          q.z = e4m3x4_q(f2.x * inv2, f2.y * inv2, f2.z * inv2, f2.w * inv2);
+          q.w = e4m3x4_q(f3.x * inv2, f3.y * inv2, f3.z * inv2, f3.w * inv2);
+          dst[v] = q;
+        }
+        fence_proxy_async_global();  // these codes are read by TMA (the async proxy)
+        quant_warps_sync();
+        if (qt == 0) red_release_gpu_add(a.q_ready + c, 1);
+      }
     }
   }
 
@@ -561,13 +684,13 @@ int resident_pairs(const cudaLaunchConfig_t& cfg, int num_sms) {
   return cache[dev];
 }
 
-template <bool kFp8, int kGemm>
+template <bool kFp8, int kGemm, bool kQuant = false>
 cudaError_t launch_pair(const GemmArgs& a, int num_sms, cudaStream_t s) {
-  constexpr auto kernel = gemm_pair_kernel<kFp8, kGemm>;
-  cudaError_t err = set_max_dynamic_smem<gemm_pair_kernel<kFp8, kGemm>>(static_cast<int>(kDynSmem));
+  constexpr auto kernel = gemm_pair_kernel<kFp8, kGemm, kQuant>;
+  cudaError_t err = set_max_dynamic_smem<gemm_pair_kernel<kFp8, kGemm, kQuant>>(static_cast<int>(kDynSmem));
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kQuant ? kQuantThreads : kThreads);
   cfg.dynamicSmemBytes = kDynSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -580,7 +703,7 @@ cudaError_t launch_pair(const GemmArgs& a, int num_sms, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.gridDim = dim3(2);
-  const int pairs = resident_pairs<gemm_pair_kernel<kFp8, kGemm>>(cfg, num_sms);
+  const int pairs = resident_pairs<gemm_pair_kernel<kFp8, kGemm, kQuant>>(cfg, num_sms);
   cfg.gridDim = dim3(2 * pairs);
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
   err = cudaLaunchKernelEx(&cfg, kernel, a);
@@ -590,6 +713,7 @@ cudaError_t launch_pair(const GemmArgs& a, int num_sms, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, bool fp8, int gemm, int num_sms, cudaStream_t s) {
+  if (fp8 && gemm == 2 && a.fuse_quant) return launch_pair<true, 2, true>(a, num_sms, s);
   if (fp8) return gemm == 1 ? launch_pair<true, 1>(a, num_sms, s) : launch_pair<true, 2>(a, num_sms, s);
   return gemm == 1 ? launch_pair<false, 1>(a, num_sms, s) : launch_pair<false, 2>(a, num_sms, s);
 }

@@ -74,6 +74,8 @@ __device__ void build_plan(const int* offsets, int E, int R, const PlanParams& p
     }
     cb += nch[j];
   }
+  if (p.ready != nullptr)  // counters of the second contraction's in-kernel quantisation
+    for (int i = lane; i < p.max_chunks; i += 32) p.ready[i] = 0;
   if (lane == 0) {
     const int nc = min(total, p.max_chunks);
     hdr->n_chunks = nc;

@@ -54,7 +54,7 @@ __device__ __forceinline__ float sigmoid_f64(float l) {
 // is [TB][E] (and [TB][E] of grouped selection scores after it) in shared memory; when
 // the experts are split over CTAs the tile's logits are in a.logits_g.  The dynamic
 // shared memory from `smem` on is reused by the permutation.
-template <int TB>
+template <int TB, int NTHR = kRouterThreads>
 __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, int tile,
                             bool split) {
   __shared__ int is_last;
@@ -77,7 +77,7 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
     }
     __syncthreads();
     if (!is_last) return;
-    for (int i = threadIdx.x; i < TB * E; i += kRouterThreads) {
+    for (int i = threadIdx.x; i < TB * E; i += NTHR) {
       const int t = i / E, e = i % E;
       logits[i] = (t0 + t < a.T) ? __ldcg(a.logits_g + static_cast<size_t>(t0 + t) * E + e) : 0.f;
     }
@@ -87,7 +87,7 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
   // ---- top-k, one warp per token
   const bool grouped = a.mode == 1;
   float* sbs = logits + TB * E;  // grouped: selection scores [TB][E]
-  for (int t = warp; t < TB; t += kRouterThreads / 32) {
+  for (int t = warp; t < TB; t += NTHR / 32) {
     const int tok = t0 + t;
     if (tok >= a.T) break;
     constexpr int kPer = kMaxExperts / 32;
@@ -207,11 +207,10 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
     // reuse: wc[8*Ea], cnt[Ea], base[Ea+1] over all Ea experts (shared ones included)
     const int Ea = a.perm.E;
     int* ps = reinterpret_cast<int*>(smem);
-    permute_body<kRouterThreads / 32>(a.perm, ps, ps + (kRouterThreads / 32) * Ea,
-                                      ps + (kRouterThreads / 32 + 1) * Ea);
+    permute_body<NTHR / 32>(a.perm, ps, ps + (NTHR / 32) * Ea, ps + (NTHR / 32 + 1) * Ea);
     if (a.fuse_gather) {
       __syncthreads();
-      gather_rows(a.gather, warp, kRouterThreads / 32);
+      gather_rows(a.gather, warp, NTHR / 32);
     }
   }
 }
@@ -336,6 +335,241 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
   router_tail<TB>(a, smem, logits, tile, split);
 }
 
+// ------------------------------------------------------------------------------------
+// Tiled router for large T*E
+//
+// One CTA computes the logits of TBC tokens x ECC experts.  Their x rows and router rows
+// stream through shared memory in slices of 256 columns, loaded by TMA into a ring of
+// kRtStages stages (one elected thread issues two tensor copies per slice), so no warp
+// waits on L2 latency.  A slice holds exactly one 8-column chunk per lane and row: lane l
+// reads chunk l of every row it needs, and over the slices in ascending order it adds the
+// chunks l, l+32, l+64, ... of each row, element by element -- the canonical order.
+// Warp w owns TBW tokens x 8 experts of the tile, one fp32 accumulator per pair and lane,
+// updated with paired FMAs (each half rounds like a scalar FMA; bf16 products are exact).
+// The 32 lane partials of a logit are combined by the xor butterfly 16, 8, 4, 2, 1 for 32
+// logits at once by recursive halving: at each step a lane keeps the half of its logits
+// whose index bit equals its lane bit and adds the partner lane's partial of the same
+// logit -- the same two operands the plain butterfly adds (fp32 addition commutes) -- so
+// logit j ends in lane j holding exactly the plain butterfly's value, after 31 shuffles
+// instead of 160.  Max |x| (CTAs of expert group 0) is taken on the bf16 bit patterns,
+// which order like the magnitudes once the sign is cleared.  The tail (expert groups
+// handed to the token tile's last CTA, top-k, weights, fused permutation) is router_tail.
+// ------------------------------------------------------------------------------------
+constexpr int kRtStages = 8;
+constexpr int kRtSlice = 256;                 // columns per slice
+constexpr int kRtRowBytes = kRtSlice * 2;     // bf16
+constexpr uint64_t kRtBudgetNs = 2000000000ull;
+constexpr int kRtLogitsOff = 32 * 1024;       // logits after the permutation scratch
+
+template <int N>
+__device__ __forceinline__ void halve(float (&v)[32], int lane) {
+  constexpr int off = N / 2;
+  const bool upper = (lane & off) != 0;
+#pragma unroll
+  for (int i = 0; i < off; ++i) {
+    const float send = upper ? v[i] : v[i + off];
+    const float keep = upper ? v[i + off] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
+}
+
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+template <int TBC, int ECC>
+constexpr size_t rt_stage_bytes() { return static_cast<size_t>(TBC + ECC) * kRtRowBytes; }
+
+// Warps of the tiled router: (ECC / 8) expert groups x as many token groups as give each
+// warp 4 tokens, i.e. 32 accumulators per lane.
+template <int TBC, int ECC>
+constexpr int rt_warps() { return (ECC / 8) * (TBC / 4); }
+
+template <int TBC, int ECC>
+__global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
+    router_tiled_kernel(const __grid_constant__ RouterArgs a, const __grid_constant__ RouterMaps m) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kRtStages];
+  __shared__ __align__(8) uint64_t empty[kRtStages];
+  __shared__ int abort_flag;
+  __shared__ uint32_t amax_bits;
+  constexpr int NW = rt_warps<TBC, ECC>();
+  constexpr int NTHR = NW * 32;
+  constexpr int NG = ECC / 8;        // groups of 8 experts in the tile
+  constexpr int TBW = 4;             // tokens per warp
+  static_assert(NG * (TBC / TBW) == NW, "warp tiling");
+  constexpr uint32_t kStageBytes = static_cast<uint32_t>(rt_stage_bytes<TBC, ECC>());
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, group = blockIdx.y;
+  const int t0 = tile * TBC, e0 = group * ECC;
+  const int tg = warp / NG, eg = warp % NG;
+  const bool split = gridDim.y > 1;
+  const int nslices = a.H / kRtSlice;
+  int32_t* status = &a.hdr->status;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kRtStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], NW);
+    }
+    abort_flag = 0;
+    amax_bits = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&m.x);
+    tma_prefetch_desc(&m.wr);
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+
+  const uint64_t pol = policy_evict_last();  // x rows and router rows are re-read by other CTAs
+  auto issue = [&](int sl) {
+    const int st = sl % kRtStages;
+    uint8_t* dst = smem + st * kStageBytes;
+    mbar_arrive_expect_tx(&full[st], kStageBytes);
+    tma_load_2d(dst, &m.x, &full[st], sl * kRtSlice, t0, pol);
+    tma_load_2d(dst + TBC * kRtRowBytes, &m.wr, &full[st], sl * kRtSlice, e0, pol);
+  };
+  int issued = 0;  // slices whose copies thread 0 started
+  if (threadIdx.x == 0) {
+    for (; issued < kRtStages && issued < nslices; ++issued) issue(issued);
+  }
+
+  float acc[TBW][8];
+#pragma unroll
+  for (int t = 0; t < TBW; ++t)
+#pragma unroll
+    for (int g = 0; g < 8; ++g) acc[t][g] = 0.f;
+  const bool do_amax = group == 0 && eg == 0;
+  uint32_t xmax = 0;  // two bf16 magnitudes, as bit patterns
+  bool ok = true;
+  for (int sl = 0; sl < nslices; ++sl) {
+    const int st = sl % kRtStages;
+    if (ok) ok = mbar_wait(&full[st], static_cast<uint32_t>((sl / kRtStages) & 1), &abort_flag, status,
+                           kRtBudgetNs);
+    if (ok) {
+      const uint8_t* xs = smem + st * kStageBytes + (tg * TBW) * kRtRowBytes;
+      const uint8_t* ws = smem + st * kStageBytes + (TBC + eg * 8) * kRtRowBytes;
+      uint4 xv[TBW], wv[8];
+#pragma unroll
+      for (int t = 0; t < TBW; ++t) xv[t] = reinterpret_cast<const uint4*>(xs + t * kRtRowBytes)[lane];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) wv[g] = reinterpret_cast<const uint4*>(ws + g * kRtRowBytes)[lane];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp has read the stage
+      if (do_amax) {
+#pragma unroll
+        for (int t = 0; t < TBW; ++t)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xmax = __vmaxu2(xmax, word_of(xv[t], q) & 0x7FFF7FFFu);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float xf[TBW], wf[8];
+#pragma unroll
+        for (int t = 0; t < TBW; ++t) {
+          const uint32_t w = word_of(xv[t], i >> 1);
+          xf[t] = (i & 1) ? hi_bf16(w) : lo_bf16(w);
+        }
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t w = word_of(wv[g], i >> 1);
+          wf[g] = (i & 1) ? hi_bf16(w) : lo_bf16(w);
+        }
+#pragma unroll
+        for (int t = 0; t < TBW; ++t)
+#pragma unroll
+          for (int g = 0; g < 8; g += 2) {
+            const float2 r = __ffma2_rn(make_float2(xf[t], xf[t]), make_float2(wf[g], wf[g + 1]),
+                                        make_float2(acc[t][g], acc[t][g + 1]));
+            acc[t][g] = r.x;
+            acc[t][g + 1] = r.y;
+          }
+      }
+    }
+    // refill: slice `issued` goes into the stage slice issued - kRtStages used, once every
+    // warp has read that slice
+    if (threadIdx.x == 0 && ok && issued < nslices && issued <= sl + kRtStages) {
+      const int old = issued - kRtStages;
+      if (mbar_wait(&empty[old % kRtStages], static_cast<uint32_t>((old / kRtStages) & 1), &abort_flag,
+                    status, kRtBudgetNs))
+        issue(issued++);
+      else
+        ok = false;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) {
+    // aborted: let the copies in flight land before the CTA exits
+    int dummy = 0;
+    for (int sl = issued > kRtStages ? issued - kRtStages : 0; sl < issued; ++sl)
+      mbar_wait(&full[sl % kRtStages], static_cast<uint32_t>((sl / kRtStages) & 1), &dummy, status,
+                kRtBudgetNs);
+  }
+  __syncthreads();
+  if (abort_flag) return;
+
+  // ---- max |x| of this token tile (expert group 0)
+  if (do_amax) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) xmax = __vmaxu2(xmax, __shfl_xor_sync(0xffffffffu, xmax, off));
+    if (lane == 0) atomicMax(&amax_bits, max(xmax & 0xFFFFu, xmax >> 16));
+  }
+
+  // ---- butterfly over lanes for the warp's 32 logits, into smem or the split buffer
+  float* logits = reinterpret_cast<float*>(smem + kRtLogitsOff);  // [TBC][E] (+ scores)
+  const int e_end = min(a.E, e0 + ECC);
+  {
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = acc[j / 8][j % 8];
+    halve<32>(v, lane);
+    halve<16>(v, lane);
+    halve<8>(v, lane);
+    halve<4>(v, lane);
+    halve<2>(v, lane);
+    const int tl = tg * TBW + lane / 8;  // token within the tile
+    const int e = e0 + eg * 8 + (lane & 7);
+    if (e < e_end) {
+      if (split) {
+        if (t0 + tl < a.T) a.logits_g[static_cast<size_t>(t0 + tl) * a.E + e] = v[0];
+      } else {
+        logits[tl * a.E + e] = v[0];
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && group == 0) {
+    a.amax_part[tile] = __uint_as_float(amax_bits << 16);
+    if (tile == 0) a.hdr->router_ctas = gridDim.x;
+  }
+  router_tail<TBC, NTHR>(a, smem, logits, tile, split);
+}
+
+template <int TBC, int ECC>
+cudaError_t launch_tiled(const RouterArgs& a0, const RouterMaps& m, cudaStream_t s) {
+  RouterArgs a = a0;
+  constexpr int NTHR = rt_warps<TBC, ECC>() * 32;
+  constexpr size_t ring = kRtStages * rt_stage_bytes<TBC, ECC>();
+  const size_t need = kRtLogitsOff + static_cast<size_t>(TBC) * a.E * 4 * 2;
+  if (a.fuse_permute) {  // permute_body's scratch sits below the logits
+    const size_t perm = static_cast<size_t>(NTHR / 32 + 2) * a.perm.E * 4 + 4;
+    if (perm > kRtLogitsOff) return cudaErrorInvalidValue;  // cannot happen: E_all <= 264
+  }
+  const size_t smem = 1024 + (ring > need ? ring : need);
+  cudaError_t err = set_max_dynamic_smem<router_tiled_kernel<TBC, ECC>>(static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int tiles = (a.T + TBC - 1) / TBC;
+  const int groups = (a.E + ECC - 1) / ECC;
+  a.experts_per_cta = groups == 1 ? a.E : ECC;
+  return launch_k(router_tiled_kernel<TBC, ECC>, dim3(tiles, groups), dim3(NTHR), smem, s, a, m);
+}
+
 template <int TB, int EG>
 cudaError_t launch_tb(RouterArgs a, cudaStream_t s) {
   size_t smem = static_cast<size_t>(TB) * a.H * 2 + static_cast<size_t>(TB) * a.E * 4 * (a.mode == 1 ? 2 : 1);
@@ -378,6 +612,20 @@ int router_tokens_per_cta(int T, int H, int E, int num_sms) {
     if (ctas >= 2L * num_sms) return tb;
   }
   return 1;
+}
+
+int router_tile_tokens(int E) { return E <= 8 ? 32 : 16; }
+int router_tile_experts(int E) { return E <= 8 ? 8 : 32; }
+
+bool router_use_tiled(int T, int E, int num_sms) {
+  const long tiles = static_cast<long>((T + router_tile_tokens(E) - 1) / router_tile_tokens(E));
+  const long groups = (E + router_tile_experts(E) - 1) / router_tile_experts(E);
+  return tiles * groups * 3 >= 2L * num_sms && tiles <= kRouterMaxTiles;
+}
+
+cudaError_t launch_router_tiled(const RouterArgs& a, const RouterMaps& m, cudaStream_t s) {
+  if (a.E <= 8) return launch_tiled<32, 8>(a, m, s);
+  return launch_tiled<16, 32>(a, m, s);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {

@@ -56,6 +56,24 @@ def max_rel_err(got, ref) -> float:
     return float(np.abs(got - ref).max() / denom)
 
 
+def per_element_err(got, ref) -> float:
+    """Per-element relative error max |got - ref| / (|ref| + 1e-3 * rms(ref)), reported for
+    information beside the normwise bound (it is not a pass/fail bar)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    return float((np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms + 1e-300)).max()) if ref.size else 0.0
+
+
+# (test id, normwise max relative error, per-element error) of every layer parity check in
+# this session; printed at the end of the run (conftest.pytest_terminal_summary)
+ERROR_REPORT = []
+
+
+def report_errors(name: str, got, ref) -> None:
+    ERROR_REPORT.append((name, max_rel_err(got, ref), per_element_err(got, ref)))
+
+
 def tiny_shape(T, H, I, E, k, wdtype, **kw):
     return minp.MoEShape(T=T, H=H, I=I, E=E, top_k=k, wdtype=wdtype, **kw)
 

@@ -120,11 +120,15 @@ def test_launch_counts():
     assert capi.fused_moe_launches_per_call(dims(k=9)) == -1
     # gathered rows above 128 KB: the gather is its own launch
     assert capi.fused_moe_launches_per_call(dims(T=256, E=8, k=2)) == 7
-    # more than 2048 routed rows: permute and gather are their own launches (normal variant)
-    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2)) == 7
-    # the CTA-pair kernels launch once per contraction like the one-CTA ones
-    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal_pair")) == 5
-    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2, variant="normal_pair")) == 7
+    # more than 2048 routed rows: permute and gather are their own launches (AUTO picks the
+    # CTA pairs here, whose FP8 second contraction quantises h itself)
+    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2)) == 6
+    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2, variant="normal")) == 7
+    # the CTA-pair kernels launch once per contraction like the one-CTA ones, and the FP8
+    # second contraction quantises h itself (no quant_h launch)
+    assert capi.fused_moe_launches_per_call(dims(T=4, variant="normal_pair")) == 4
+    assert capi.fused_moe_launches_per_call(dims(T=2048, E=8, k=2, variant="normal_pair")) == 6
+    assert capi.fused_moe_launches_per_call(dims(T=4, fp8=False, variant="normal_pair")) == 4
 
 
 def test_shared_expert_validation_and_workspace():
@@ -275,8 +279,12 @@ def test_host_properties_over_many_dims():
             assert capi.workspace_size(d) >= R * H * (es + 4) + R * I * es
             # variant the library resolves for AUTO: <= 64 rows per expert on average ->
             # swap-AB, else the normal tiles (one CTA or pairs)
-            swap = variant == "swap_ab" or (variant == "auto" and (R + E + ns - 1) // (E + ns) <= 64)
-            n = 4 + (1 if fp8 else 0) + (1 if swap else 0)
+            avg = (R + E + ns - 1) // (E + ns)
+            swap = variant == "swap_ab" or (variant == "auto" and avg <= 64)
+            pair = variant == "normal_pair" or (variant == "auto" and avg > 128)
+            # quant_h runs as its own launch in the FP8 format, except that the CTA-pair
+            # second contraction quantises h itself
+            n = 4 + (1 if fp8 and not pair else 0) + (1 if swap else 0)
             if R > 2048:
                 n += 2
             elif R * H * 2 > 128 * 1024:

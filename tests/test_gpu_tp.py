@@ -13,7 +13,7 @@ import torch
 
 from oracle import fused_moe_oracle as O
 from mixture_experts_layer_26_b200 import inputs as minp
-from helpers import run_oracle, max_rel_err, bf16_bits_to_float, tiny_shape
+from helpers import run_oracle, max_rel_err, bf16_bits_to_float, tiny_shape, report_errors
 
 capi = pytest.importorskip("mixture_experts_layer_26_b200.capi")
 from mixture_experts_layer_26_b200 import tp  # noqa: E402
@@ -110,6 +110,7 @@ def test_shards_match_the_unsharded_oracle(small, name, shape, kw, n, variant):
     wd = inp.shape.wdtype
     bits, gmax, local = run_tp(inp, g, n, variant)
     err = max_rel_err(bf16_bits_to_float(bits), ref["out64"])
+    report_errors(f"tp {name} N={n} {variant}", bf16_bits_to_float(bits), ref["out64"])
     assert err <= TOL[wd], err
     if wd == "fp8":
         _, amax_unsharded = run_unsharded(inp, g, variant)
@@ -145,6 +146,7 @@ def test_full_size_shards_match_oracle(workload, T, n):
     ref = run_oracle(O, inp)
     bits, gmax, _ = run_tp(inp, g, n)
     err = max_rel_err(bf16_bits_to_float(bits), ref["out64"])
+    report_errors(f"tp {workload} T={T} N={n}", bf16_bits_to_float(bits), ref["out64"])
     assert err <= TOL[s.wdtype], err
     if s.wdtype == "fp8":
         assert abs(gmax / float(np.abs(ref["h"]).max()) - 1) <= 1e-5
