@@ -614,15 +614,31 @@ __global__ void __launch_bounds__(kQuant ? kQuantThreads : kThreads, 1)
         const size_t v0 = min(n16, blockIdx.x * per), v1 = min(n16, v0 + per);
         const float4* src = reinterpret_cast<const float4*>(a.q_h + base);
         uint4* dst = reinterpret_cast<uint4*>(a.q_hq + base);
-        for (size_t v = v0 + qt; v < v1; v += 128) {
-          const float4 f0 = __ldcs(src + 4 * v), f1 = __ldcs(src + 4 * v + 1);
-          const float4 f2 = __ldcs(src + 4 * v + 2), f3 = __ldcs(src + 4 * v + 3);
-          uint4 q;
-          q.x = e4m3x4_q(f0.x * inv2, f0.y * inv2, f0.z * inv2, f0.w * inv2);
-          q.y = e4m3x4_q(f1.x * inv2, f1.y * inv2, f1.z * inv2, f1.w * inv2);
-          q.z = e4m3x4_q(f2.x * inv2, f2.y * inv2, f2.z * inv2, f2.w * inv2);
-          q.w = e4m3x4_q(f3.x * inv2, f3.y * inv2, f3.z * inv2, f3.w * inv2);
-          dst[v] = q;
+        // kQU vectors of 16 values per thread in flight (256 bytes), so that 128 threads
+        // per SM keep enough loads outstanding to stream h near HBM speed
+        constexpr int kQU = 4;
+        for (size_t v = v0 + qt; v < v1; v += 128 * kQU) {
+          float4 f[kQU][4];
+#pragma unroll
+          for (int u = 0; u < kQU; ++u) {
+            const size_t w = v + 128 * u;
+            if (w < v1) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) f[u][j] = __ldcs(src + 4 * w + j);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kQU; ++u) {
+            const size_t w = v + 128 * u;
+            if (w < v1) {
+              uint4 q;
+              q.x = e4m3x4_q(f[u][0].x * inv2, f[u][0].y * inv2, f[u][0].z * inv2, f[u][0].w * inv2);
+              q.y = e4m3x4_q(f[u][1].x * inv2, f[u][1].y * inv2, f[u][1].z * inv2, f[u][1].w * inv2);
+              q.z = e4m3x4_q(f[u][2].x * inv2, f[u][2].y * inv2, f[u][2].z * inv2, f[u][2].w * inv2);
+              q.w = e4m3x4_q(f[u][3].x * inv2, f[u][3].y * inv2, f[u][3].z * inv2, f[u][3].w * inv2);
+              dst[w] = q;
+            }
+          }
         }
         fence_proxy_async_global();  // these codes are read by TMA (the async proxy)
         quant_warps_sync();

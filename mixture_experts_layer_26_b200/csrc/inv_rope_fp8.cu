@@ -73,7 +73,12 @@ __device__ __forceinline__ void load_row(const float* p, float (&v)[N]) {
 // of x per step.
 template <int EPL> constexpr int heads_per_step() { return EPL == 8 ? 4 : 8; }
 
-template <int EPL, int kStyle>
+// Two lanes' worth of arithmetic per instruction: Blackwell's paired fp32 multiply and add
+// round each half exactly like the scalar __fmul_rn / __fadd_rn.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+template <int EPL, int kStyle, bool kFull>
 __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeArgs a) {
   griddep_wait();
   griddep_launch_dependents();
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
   const int nwarps = (gridDim.x * kRopeThreads) >> 5;
   const int hd = 32 * EPL, rot = a.rot_dim, half = rot / 2;
   const int j0 = lane * EPL;               // first coordinate of this lane
-  const bool rotated = j0 < rot;           // EPL divides rot: a lane is all in or all out
+  const bool rotated = kFull || j0 < rot;  // EPL divides rot: a lane is all in or all out
   const bool is_a = kStyle == 0 ? j0 < half : true;
   // style 0: pair index of coordinate j0 (its partner's too); style 1: j0 / 2
   const int i0 = kStyle == 0 ? (is_a ? j0 : j0 - half) : j0 / 2;
@@ -159,12 +164,15 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
     const int p_after = pos_of(ua);
 
     const int h0 = uc.hg * HPS;
-    uint8_t* qdst = a.q + (static_cast<size_t>(uc.t) * a.n_heads + h0) * hd + j0;
-    float* sdst = a.scales + static_cast<size_t>(uc.t) * a.n_heads + h0;
+    const int nh = min(HPS, a.n_heads - h0);  // heads of this unit (warp-uniform)
+    // ---- rotate every head of the unit and take its max |y| (warp-uniform m[k])
+    float y[HPS][EPL];
+    float m[HPS];
 #pragma unroll
     for (int k = 0; k < HPS; ++k) {
-      if (h0 + k >= a.n_heads) break;  // warp-uniform
-      float x[EPL], y[EPL];
+      m[k] = 0.f;
+      if (k >= nh) continue;
+      float x[EPL];
       unpack_bf16<EPL>(xc[k], x);
       if constexpr (kStyle == 0) {
         // the partner's coordinates, moved as packed bf16 pairs (one shuffle per word)
@@ -177,35 +185,51 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
           o[2 * i + 1] = __uint_as_float(ow & 0xFFFF0000u);
         }
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          const float r = __fadd_rn(__fmul_rn(x[e], cc[e]), __fmul_rn(o[e], sc_[e]));
-          y[e] = rotated ? r : x[e];
+        for (int e = 0; e < EPL; e += 2) {
+          const float2 r = add2(mul2(make_float2(x[e], x[e + 1]), make_float2(cc[e], cc[e + 1])),
+                                mul2(make_float2(o[e], o[e + 1]), make_float2(sc_[e], sc_[e + 1])));
+          y[k][e] = rotated ? r.x : x[e];
+          y[k][e + 1] = rotated ? r.y : x[e + 1];
         }
       } else {
 #pragma unroll
         for (int e = 0; e < EPL; e += 2) {
           const float c = cc[e / 2], sn = sc_[e / 2];
-          const float r0 = __fadd_rn(__fmul_rn(x[e], c), __fmul_rn(x[e + 1], sn));
-          const float r1 = __fadd_rn(__fmul_rn(x[e + 1], c), __fmul_rn(x[e], -sn));
-          y[e] = rotated ? r0 : x[e];
-          y[e + 1] = rotated ? r1 : x[e + 1];
+          const float2 r = add2(mul2(make_float2(x[e], x[e + 1]), make_float2(c, c)),
+                                mul2(make_float2(x[e + 1], x[e]), make_float2(sn, -sn)));
+          y[k][e] = rotated ? r.x : x[e];
+          y[k][e + 1] = rotated ? r.y : x[e + 1];
         }
       }
-      // max |y| over the head: the bit patterns of non-negative finite floats order like
-      // unsigned integers, so one warp-wide unsigned max gives it exactly
-      uint32_t mb = 0;
+      // max |y| over the head: non-negative finite floats order like their bit patterns,
+      // so a warp-wide unsigned max of the lane maxima gives it exactly
+      float mx = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) mb = max(mb, __float_as_uint(y[e]) & 0x7FFFFFFFu);
-      const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, mb));
-      const float inv = m > 0.f ? 448.0f / m : 1.f;
+      for (int e = 0; e < EPL; ++e) mx = fmaxf(mx, fabsf(y[k][e]));
+      m[k] = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+    }
+    // ---- the unit's scales, head k on lane k: one IEEE division each for the inverse
+    // scale 448/m and the scale m/448 (1 for an all-zero head)
+    float ml = 0.f;
+#pragma unroll
+    for (int k = 0; k < HPS; ++k) ml = lane == k ? m[k] : ml;
+    const float inv_l = ml > 0.f ? 448.0f / ml : 1.f;
+    const float scale_l = ml > 0.f ? ml / 448.0f : 1.f;
+    if (lane < nh) __stcs(a.scales + static_cast<size_t>(uc.t) * a.n_heads + h0 + lane, scale_l);
+    // ---- quantise and store
+    uint8_t* qdst = a.q + (static_cast<size_t>(uc.t) * a.n_heads + h0) * hd + j0;
+#pragma unroll
+    for (int k = 0; k < HPS; ++k) {
+      if (k >= nh) break;  // warp-uniform
+      const float inv = __shfl_sync(0xffffffffu, inv_l, k);
       typename Vec<EPL>::Q qv;
       uint16_t* q16 = reinterpret_cast<uint16_t*>(&qv);
 #pragma unroll
-      for (int e = 0; e < EPL; e += 2)
-        q16[e / 2] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(
-            make_float2(__fmul_rn(y[e], inv), __fmul_rn(y[e + 1], inv)), __NV_SATFINITE, __NV_E4M3));
+      for (int e = 0; e < EPL; e += 2) {
+        const float2 p = mul2(make_float2(y[k][e], y[k][e + 1]), make_float2(inv, inv));
+        q16[e / 2] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(p, __NV_SATFINITE, __NV_E4M3));
+      }
       __stcs(reinterpret_cast<typename Vec<EPL>::Q*>(qdst + k * hd), qv);
-      if (lane == 0) __stcs(sdst + k, m > 0.f ? m / 448.0f : 1.f);
     }
 #pragma unroll
     for (int k = 0; k < HPS; ++k) xc[k] = xn[k];
@@ -221,7 +245,7 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
   }
 }
 
-template <int EPL, int kStyle>
+template <int EPL, int kStyle, bool kFull>
 cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
   constexpr int HPS = heads_per_step<EPL>();
   const long units = static_cast<long>(a.T) * ((a.n_heads + HPS - 1) / HPS);  // < 2^31
@@ -232,7 +256,7 @@ cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   if (resident[dev] == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, inv_rope_fp8_kernel<EPL, kStyle>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, inv_rope_fp8_kernel<EPL, kStyle, kFull>,
                                                       kRopeThreads, 0) != cudaSuccess || n < 1) {
       (void)cudaGetLastError();
       n = 1;
@@ -242,22 +266,29 @@ cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
   const long cap = static_cast<long>(num_sms) * resident[dev];
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  return launch_k(inv_rope_fp8_kernel<EPL, kStyle>, dim3(static_cast<unsigned>(grid)),
+  return launch_k(inv_rope_fp8_kernel<EPL, kStyle, kFull>, dim3(static_cast<unsigned>(grid)),
                   dim3(kRopeThreads), 0, s, a);
 }
 
 }  // namespace
 
+template <int EPL, int kStyle>
+cudaError_t launch_rope_rot(const RopeArgs& a, int num_sms, cudaStream_t s) {
+  // every coordinate rotated (the usual full rotary): no pass-through selects
+  if (a.rot_dim == a.head_dim) return launch_rope<EPL, kStyle, true>(a, num_sms, s);
+  return launch_rope<EPL, kStyle, false>(a, num_sms, s);
+}
+
 cudaError_t launch_inv_rope_fp8(const RopeArgs& a, int num_sms, cudaStream_t s) {
   const int epl = a.head_dim / 32;
   if (a.style == 0) {
-    if (epl == 2) return launch_rope<2, 0>(a, num_sms, s);
-    if (epl == 4) return launch_rope<4, 0>(a, num_sms, s);
-    return launch_rope<8, 0>(a, num_sms, s);
+    if (epl == 2) return launch_rope_rot<2, 0>(a, num_sms, s);
+    if (epl == 4) return launch_rope_rot<4, 0>(a, num_sms, s);
+    return launch_rope_rot<8, 0>(a, num_sms, s);
   }
-  if (epl == 2) return launch_rope<2, 1>(a, num_sms, s);
-  if (epl == 4) return launch_rope<4, 1>(a, num_sms, s);
-  return launch_rope<8, 1>(a, num_sms, s);
+  if (epl == 2) return launch_rope_rot<2, 1>(a, num_sms, s);
+  if (epl == 4) return launch_rope_rot<4, 1>(a, num_sms, s);
+  return launch_rope_rot<8, 1>(a, num_sms, s);
 }
 
 }  // namespace fmoe

@@ -53,6 +53,8 @@ SMALL = [
     (13, 4, 64, 64, 1),
     (9, 1, 256, 128, 1),
     (1, 1, 128, 8, 0),      # one token, one head, the shortest rotary span for 128
+    (21, 9, 128, 128, 1),   # interleaved, full rotary, a second head group of one head
+    (15, 12, 64, 64, 0),    # half split, full rotary, head groups of eight and four
 ]
 
 
