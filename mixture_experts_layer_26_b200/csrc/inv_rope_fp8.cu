@@ -17,12 +17,14 @@
 //
 // HBM-bound: 2 bytes read and 1 byte written per element plus 4 bytes of scale per
 // head; the rotary table (max_pos x rot_dim fp32) is gathered through L2.  One warp
-// handles up to eight heads of one token per step, lane l owning the EPL = head_dim/32
+// handles units of up to four heads of one token, lane l owning the EPL = head_dim/32
 // consecutive coordinates [EPL*l, EPL*l + EPL) of each head: one vector load and one
-// packed store per head and lane, with the next step's loads in flight meanwhile.  The
+// packed store per head and lane, with the next unit's loads in flight meanwhile.  The
 // half-split partner of a coordinate lives rot_dim/(2*EPL) lanes away (a lane xor for
-// power-of-two rot_dim); interleaved partners are in the same lane.  The grid is the
-// number of blocks that fit on the GPU at once (a persistent grid-stride loop).
+// power-of-two rot_dim); interleaved partners are in the same lane.  A unit's scales are
+// computed one head per lane (two IEEE divisions per head, issued once per unit) and
+// broadcast by shuffles.  The grid is the number of blocks that fit on the GPU at once
+// (a persistent grid-stride loop).
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -69,33 +71,122 @@ __device__ __forceinline__ void load_row(const float* p, float (&v)[N]) {
   }
 }
 
-// Heads a warp takes per step: 8 (4 for head_dim 256), so that each lane keeps 32 bytes
-// of x per step.
-template <int EPL> constexpr int heads_per_step() { return EPL == 8 ? 4 : 8; }
+// Heads a warp takes per unit: 4, so that the registers of a unit in flight and of the
+// next one stay small enough for three 256-thread blocks per SM (two for head_dim 256).
+template <int EPL> constexpr int heads_per_step() { return 4; }
 
-// Two lanes' worth of arithmetic per instruction: Blackwell's paired fp32 multiply and add
-// round each half exactly like the scalar __fmul_rn / __fadd_rn.
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// fadd(fmul(x, c), fmul(o, s)) for two coordinates, each product and each sum rounded
+// separately (__fmul_rn / __fadd_rn are never contracted into a fused multiply-add).  The
+// paired fp32 instructions were tried here and changed the last bit of some results, so
+// the scalar forms stay.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+}
+__device__ __forceinline__ float2 rot2(float2 x, float2 c, float2 o, float2 s) {
+  return make_float2(__fadd_rn(__fmul_rn(x.x, c.x), __fmul_rn(o.x, s.x)),
+                     __fadd_rn(__fmul_rn(x.y, c.y), __fmul_rn(o.y, s.y)));
+}
 
 template <int EPL, int kStyle, bool kFull>
-__global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeArgs a) {
+__device__ __forceinline__ void rope_unit(const typename Vec<EPL>::X (&xv)[heads_per_step<EPL>()],
+                                          int nh, const float* cc, const float* sn, bool rotated,
+                                          int partner_xor, int lane, uint8_t* qdst, int hd,
+                                          float* sdst) {
+  constexpr int HPS = heads_per_step<EPL>();
+  constexpr int NW = EPL / 2;  // 32-bit words (bf16 pairs) per lane
+  float y[HPS][EPL];
+  float m[HPS];
+#pragma unroll
+  for (int k = 0; k < HPS; ++k) {
+    m[k] = 0.f;
+    if (k >= nh) continue;  // warp-uniform
+    float x[EPL];
+    unpack_bf16<EPL>(xv[k], x);
+    if constexpr (kStyle == 0) {
+      // the partner's coordinates, moved as packed bf16 pairs (one shuffle per word)
+      const uint32_t* wv = reinterpret_cast<const uint32_t*>(&xv[k]);
+      float o[EPL];
+#pragma unroll
+      for (int i = 0; i < NW; ++i) {
+        const uint32_t ow = __shfl_xor_sync(0xffffffffu, wv[i], partner_xor);
+        o[2 * i] = __uint_as_float(ow << 16);
+        o[2 * i + 1] = __uint_as_float(ow & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2) {
+        const float2 r = rot2(make_float2(x[e], x[e + 1]), make_float2(cc[e], cc[e + 1]),
+                              make_float2(o[e], o[e + 1]), make_float2(sn[e], sn[e + 1]));
+        y[k][e] = (kFull || rotated) ? r.x : x[e];
+        y[k][e + 1] = (kFull || rotated) ? r.y : x[e + 1];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2) {
+        const float c = cc[e / 2], s = sn[e / 2];
+        const float2 r = rot2(make_float2(x[e], x[e + 1]), make_float2(c, c),
+                              make_float2(x[e + 1], x[e]), make_float2(s, -s));
+        y[k][e] = (kFull || rotated) ? r.x : x[e];
+        y[k][e + 1] = (kFull || rotated) ? r.y : x[e + 1];
+      }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) mx = fmaxf(mx, fabsf(y[k][e]));
+    m[k] = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  }
+  float ml = 0.f;  // head `lane`'s max |y|
+#pragma unroll
+  for (int k = 0; k < HPS; ++k) ml = lane == k ? m[k] : ml;
+  const float inv_l = ml > 0.f ? 448.0f / ml : 1.f;
+  if (lane < nh) __stcs(sdst + lane, ml > 0.f ? ml / 448.0f : 1.f);
+#pragma unroll
+  for (int k = 0; k < HPS; ++k) {
+    if (k >= nh) break;  // warp-uniform
+    const float inv = __shfl_sync(0xffffffffu, inv_l, k);
+    typename Vec<EPL>::Q qv;
+    uint16_t* q16 = reinterpret_cast<uint16_t*>(&qv);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+      const float2 p = mul2(make_float2(y[k][e], y[k][e + 1]), make_float2(inv, inv));
+      q16[e / 2] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(p, __NV_SATFINITE, __NV_E4M3));
+    }
+    __stcs(reinterpret_cast<typename Vec<EPL>::Q*>(qdst + k * hd), qv);
+  }
+}
+
+// Lane geometry shared by both kernels.
+template <int EPL, int kStyle>
+struct RopeLane {
+  int j0, half, i0, partner_xor;
+  bool rotated, is_a;
+  __device__ RopeLane(const RopeArgs& a, int lane) {
+    const int rot = a.rot_dim;
+    half = rot / 2;
+    j0 = lane * EPL;                 // first coordinate of this lane
+    rotated = j0 < rot;              // EPL divides rot: a lane is all in or all out
+    is_a = kStyle == 0 ? j0 < half : true;
+    // style 0: pair index of coordinate j0 (its partner's too); style 1: j0 / 2
+    i0 = kStyle == 0 ? (is_a ? j0 : j0 - half) : j0 / 2;
+    partner_xor = kStyle == 0 ? half / EPL : 0;
+  }
+};
+
+// ------------------------------------------------------------------------------------
+// The kernel: each warp keeps the next unit's x rows and table entries in registers
+// while it works on the current one.
+// ------------------------------------------------------------------------------------
+template <int EPL, int kStyle, bool kFull>
+__global__ void __launch_bounds__(kRopeThreads, EPL == 8 ? 2 : 3) inv_rope_fp8_kernel(const RopeArgs a) {
   griddep_wait();
   griddep_launch_dependents();
   constexpr int HPS = heads_per_step<EPL>();
   constexpr int NC = kStyle == 0 ? EPL : EPL / 2;  // table entries a lane needs
-  constexpr int NW = EPL / 2;                      // 32-bit words (bf16 pairs) per lane
   using XV = typename Vec<EPL>::X;
   const int lane = threadIdx.x & 31;
   const int gwarp = (blockIdx.x * kRopeThreads + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * kRopeThreads) >> 5;
-  const int hd = 32 * EPL, rot = a.rot_dim, half = rot / 2;
-  const int j0 = lane * EPL;               // first coordinate of this lane
-  const bool rotated = kFull || j0 < rot;  // EPL divides rot: a lane is all in or all out
-  const bool is_a = kStyle == 0 ? j0 < half : true;
-  // style 0: pair index of coordinate j0 (its partner's too); style 1: j0 / 2
-  const int i0 = kStyle == 0 ? (is_a ? j0 : j0 - half) : j0 / 2;
-  const int partner_xor = kStyle == 0 ? half / EPL : 0;
+  const int hd = 32 * EPL, rot = a.rot_dim;
+  const RopeLane<EPL, kStyle> L(a, lane);
   const int hgroups = (a.n_heads + HPS - 1) / HPS;
   const int units = a.T * hgroups;  // < 2^31: T * n_heads * head_dim is checked on the host
 
@@ -129,7 +220,7 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
     if (w.t >= a.T) return;
     const int h0 = w.hg * HPS;
     const XV* src = reinterpret_cast<const XV*>(
-        a.x + (static_cast<size_t>(w.t) * a.n_heads + h0) * hd + j0);
+        a.x + (static_cast<size_t>(w.t) * a.n_heads + h0) * hd + L.j0);
 #pragma unroll
     for (int k = 0; k < HPS; ++k)
       if (h0 + k < a.n_heads) xv[k] = __ldcs(src + k * 32);  // streamed once
@@ -138,11 +229,11 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
   // rotated coordinate is fadd(fmul(x, cos), fmul(partner, sin')): for b that is
   // -(x_a*sin) + x_b*cos exactly (IEEE addition commutes and negation is exact)
   auto load_table = [&](Unit w, int p, float (&cs)[NC], float (&sn)[NC]) {
-    if (w.t >= a.T || !rotated) return;
+    if (w.t >= a.T || !(kFull || L.rotated)) return;
     const float* row = a.cos_sin + static_cast<size_t>(p) * rot;
-    load_row<NC>(row + i0, cs);
-    load_row<NC>(row + half + i0, sn);
-    if (kStyle == 0 && !is_a) {
+    load_row<NC>(row + L.i0, cs);
+    load_row<NC>(row + L.half + L.i0, sn);
+    if (kStyle == 0 && !L.is_a) {
 #pragma unroll
       for (int i = 0; i < NC; ++i) sn[i] = -sn[i];
     }
@@ -162,75 +253,10 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
     load_x(un, xn);
     load_table(un, p_next, cn, sn_);
     const int p_after = pos_of(ua);
-
     const int h0 = uc.hg * HPS;
-    const int nh = min(HPS, a.n_heads - h0);  // heads of this unit (warp-uniform)
-    // ---- rotate every head of the unit and take its max |y| (warp-uniform m[k])
-    float y[HPS][EPL];
-    float m[HPS];
-#pragma unroll
-    for (int k = 0; k < HPS; ++k) {
-      m[k] = 0.f;
-      if (k >= nh) continue;
-      float x[EPL];
-      unpack_bf16<EPL>(xc[k], x);
-      if constexpr (kStyle == 0) {
-        // the partner's coordinates, moved as packed bf16 pairs (one shuffle per word)
-        const uint32_t* wv = reinterpret_cast<const uint32_t*>(&xc[k]);
-        float o[EPL];
-#pragma unroll
-        for (int i = 0; i < NW; ++i) {
-          const uint32_t ow = __shfl_xor_sync(0xffffffffu, wv[i], partner_xor);
-          o[2 * i] = __uint_as_float(ow << 16);
-          o[2 * i + 1] = __uint_as_float(ow & 0xFFFF0000u);
-        }
-#pragma unroll
-        for (int e = 0; e < EPL; e += 2) {
-          const float2 r = add2(mul2(make_float2(x[e], x[e + 1]), make_float2(cc[e], cc[e + 1])),
-                                mul2(make_float2(o[e], o[e + 1]), make_float2(sc_[e], sc_[e + 1])));
-          y[k][e] = rotated ? r.x : x[e];
-          y[k][e + 1] = rotated ? r.y : x[e + 1];
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < EPL; e += 2) {
-          const float c = cc[e / 2], sn = sc_[e / 2];
-          const float2 r = add2(mul2(make_float2(x[e], x[e + 1]), make_float2(c, c)),
-                                mul2(make_float2(x[e + 1], x[e]), make_float2(sn, -sn)));
-          y[k][e] = rotated ? r.x : x[e];
-          y[k][e + 1] = rotated ? r.y : x[e + 1];
-        }
-      }
-      // max |y| over the head: non-negative finite floats order like their bit patterns,
-      // so a warp-wide unsigned max of the lane maxima gives it exactly
-      float mx = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) mx = fmaxf(mx, fabsf(y[k][e]));
-      m[k] = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
-    }
-    // ---- the unit's scales, head k on lane k: one IEEE division each for the inverse
-    // scale 448/m and the scale m/448 (1 for an all-zero head)
-    float ml = 0.f;
-#pragma unroll
-    for (int k = 0; k < HPS; ++k) ml = lane == k ? m[k] : ml;
-    const float inv_l = ml > 0.f ? 448.0f / ml : 1.f;
-    const float scale_l = ml > 0.f ? ml / 448.0f : 1.f;
-    if (lane < nh) __stcs(a.scales + static_cast<size_t>(uc.t) * a.n_heads + h0 + lane, scale_l);
-    // ---- quantise and store
-    uint8_t* qdst = a.q + (static_cast<size_t>(uc.t) * a.n_heads + h0) * hd + j0;
-#pragma unroll
-    for (int k = 0; k < HPS; ++k) {
-      if (k >= nh) break;  // warp-uniform
-      const float inv = __shfl_sync(0xffffffffu, inv_l, k);
-      typename Vec<EPL>::Q qv;
-      uint16_t* q16 = reinterpret_cast<uint16_t*>(&qv);
-#pragma unroll
-      for (int e = 0; e < EPL; e += 2) {
-        const float2 p = mul2(make_float2(y[k][e], y[k][e + 1]), make_float2(inv, inv));
-        q16[e / 2] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(p, __NV_SATFINITE, __NV_E4M3));
-      }
-      __stcs(reinterpret_cast<typename Vec<EPL>::Q*>(qdst + k * hd), qv);
-    }
+    const size_t head0 = static_cast<size_t>(uc.t) * a.n_heads + h0;
+    rope_unit<EPL, kStyle, kFull>(xc, min(HPS, a.n_heads - h0), cc, sc_, L.rotated,
+                                  L.partner_xor, lane, a.q + head0 * hd + L.j0, hd, a.scales + head0);
 #pragma unroll
     for (int k = 0; k < HPS; ++k) xc[k] = xn[k];
 #pragma unroll
@@ -248,12 +274,12 @@ __global__ void __launch_bounds__(kRopeThreads) inv_rope_fp8_kernel(const RopeAr
 template <int EPL, int kStyle, bool kFull>
 cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
   constexpr int HPS = heads_per_step<EPL>();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   const long units = static_cast<long>(a.T) * ((a.n_heads + HPS - 1) / HPS);  // < 2^31
   const long warps_per_block = kRopeThreads / 32;
   long grid = (units + warps_per_block - 1) / warps_per_block;
   static int resident[64] = {0};  // blocks per SM, per device
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   if (resident[dev] == 0) {
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, inv_rope_fp8_kernel<EPL, kStyle, kFull>,
@@ -270,14 +296,14 @@ cudaError_t launch_rope(const RopeArgs& a, int num_sms, cudaStream_t s) {
                   dim3(kRopeThreads), 0, s, a);
 }
 
-}  // namespace
-
 template <int EPL, int kStyle>
 cudaError_t launch_rope_rot(const RopeArgs& a, int num_sms, cudaStream_t s) {
   // every coordinate rotated (the usual full rotary): no pass-through selects
   if (a.rot_dim == a.head_dim) return launch_rope<EPL, kStyle, true>(a, num_sms, s);
   return launch_rope<EPL, kStyle, false>(a, num_sms, s);
 }
+
+}  // namespace
 
 cudaError_t launch_inv_rope_fp8(const RopeArgs& a, int num_sms, cudaStream_t s) {
   const int epl = a.head_dim / 32;

@@ -196,7 +196,13 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
     // activation scale from the router's per-tile maxima (one warp, strided)
     float amax = 0.f;
     const int n = __ldcg(&a.hdr->router_ctas);
-    for (int i = lane; i < n; i += 32) amax = fmaxf(amax, __ldcg(a.amax_part + i));
+    for (int i0 = lane; i0 < n; i0 += 32 * 8) {  // eight loads in flight per lane
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = i0 + 32 * j < n ? __ldcg(a.amax_part + i0 + 32 * j) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, v[j]);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     float s1 = 1.f, inv1 = 1.f;
@@ -268,10 +274,25 @@ __device__ void gather_rows(const GatherArgs& a, int gwarp, int nwarps) {
     const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
     if (a.fp8) {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);
-      for (int v = lane; v < nvec; v += 32) {
-        const uint4 x0 = __ldg(src + 2 * v), x1 = __ldg(src + 2 * v + 1);
-        const uint2 q0 = quant8(x0, inv), q1 = quant8(x1, inv);
-        dst[v] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+      constexpr int kU = 4;  // 128 bytes of x per lane in flight
+      for (int v0 = lane; v0 < nvec; v0 += 32 * kU) {
+        uint4 x0[kU], x1[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+            x0[u] = __ldg(src + 2 * v);
+            x1[u] = __ldg(src + 2 * v + 1);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+            const uint2 q0 = quant8(x0[u], inv), q1 = quant8(x1[u], inv);
+            dst[v] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+          }
+        }
       }
     } else {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);

@@ -355,11 +355,6 @@ __global__ void __launch_bounds__(kRouterThreads, 2) router_kernel(RouterArgs a)
 // which order like the magnitudes once the sign is cleared.  The tail (expert groups
 // handed to the token tile's last CTA, top-k, weights, fused permutation) is router_tail.
 // ------------------------------------------------------------------------------------
-// Paired (two-lane) FMAs in the tiled router's inner product; either form rounds each
-// product-sum exactly like a scalar fmaf, so the logits are the same bits.
-#ifndef FMOE_ROUTER_PAIRED_FMA
-#define FMOE_ROUTER_PAIRED_FMA 1
-#endif
 constexpr int kRtStages = 8;
 constexpr int kRtSlice = 256;                 // columns per slice
 constexpr int kRtRowBytes = kRtSlice * 2;     // bf16
@@ -486,7 +481,6 @@ __global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
           const uint32_t w = word_of(wv[g], i >> 1);
           wf[g] = (i & 1) ? hi_bf16(w) : lo_bf16(w);
         }
-#if FMOE_ROUTER_PAIRED_FMA
 #pragma unroll
         for (int t = 0; t < TBW; ++t)
 #pragma unroll
@@ -496,12 +490,6 @@ __global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
             acc[t][g] = r.x;
             acc[t][g + 1] = r.y;
           }
-#else
-#pragma unroll
-        for (int t = 0; t < TBW; ++t)
-#pragma unroll
-          for (int g = 0; g < 8; ++g) acc[t][g] = __fmaf_rn(xf[t], wf[g], acc[t][g]);
-#endif
       }
     }
     // refill: slice `issued` goes into the stage slice issued - kRtStages used, once every
