@@ -637,7 +637,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     s = minp.shape(args.workload, args.T)
-    L = Layer(s, dev, args.variant)
+    L = Layer(s, dev, args.variant, weights_on_device=s.E_all * s.H * s.I > 2 ** 31)
     m = measure_layer(L, args, dist, rank, world, dev)
 
     # decode regimes beside the default prefill workload, measured the same way
@@ -668,7 +668,11 @@ def run_ours(args, rank, world, local_rank):
                                                        args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_sample(L.inp, args.cpu_budget)
+        inp = L.inp
+        if inp.w13.is_cuda:  # weights drawn on the device: the oracle reads host copies
+            inp = minp.MoEInputs(s, inp.x, inp.router_w, inp.w13.cpu(), inp.w2.cpu(), inp.w13_scale,
+                                 inp.w2_scale, inp.router_bias)
+        cpu = cpu_baseline_sample(inp, args.cpu_budget)
     fp8 = s.wdtype == "fp8"
     line = {
         "metric": METRIC, "value": round(m["value"], 1), "unit": "tokens/s", "n_gpus": world,
@@ -988,7 +992,9 @@ def run_rope_ours(args, rank, world, local_rank):
             "frac": round(ach / peaks["hbm_gbs"], 4),
             "traffic": profiled_traffic(kname, f"{args.workload}_T{s.T}"),
             "kernel": kname, "kernel_us": round(1e3 * ms_launch, 2), "algorithmic_bytes": nbytes,
-            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"}
+            "peak_kind": (f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy stream)"
+                          if peak_kind == "measured" else
+                          "fallback 6650 GB/s (no MEASURED_PEAKS.json)")}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         n = min(s.T, 2048)
