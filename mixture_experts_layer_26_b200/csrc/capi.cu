@@ -74,6 +74,12 @@ fmoe_status check_dims(const fmoe_dims* d) {
   return FMOE_OK;
 }
 
+int swap_chunk_cap(const fmoe_dims& d) {
+  const bool concentrated =
+      d.routing != nullptr && (d.routing->n_shared > 0 || d.routing->mode == FMOE_ROUTE_SIGMOID_GROUPED);
+  return concentrated ? 128 : 64;
+}
+
 Layout make_layout(const fmoe_dims& d) {
   Layout L;
   L.fp8 = d.wdtype == FMOE_FP8_E4M3;
@@ -87,8 +93,10 @@ Layout make_layout(const fmoe_dims& d) {
   }
   L.swap = variant == FMOE_VARIANT_SWAP_AB;
   L.pair = variant == FMOE_VARIANT_NORMAL_PAIR;
-  // an expert receives at most T rows (one per token)
-  L.chunk_rows = L.swap ? std::min(64, static_cast<int>(align_up(std::max(T, 1), 16)))
+  // an expert receives at most T rows (one per token).  Swap-AB chunks hold up to 64 rows,
+  // or 128 when some experts are known to receive many more than the average: every token
+  // uses a shared expert, and grouped routing concentrates the batch on a few groups
+  L.chunk_rows = L.swap ? std::min(swap_chunk_cap(d), static_cast<int>(align_up(std::max(T, 1), 16)))
                         : (L.pair ? 256 : 128);
   L.max_chunks = R / L.chunk_rows + std::min(E, R) + 1;
   const size_t es = L.fp8 ? 1 : 2;

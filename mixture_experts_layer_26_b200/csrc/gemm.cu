@@ -49,11 +49,13 @@ constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 128-byte operand
 constexpr int kSwapBoxRows = 16;        // token rows per TMA box in the swap-AB variant
 // Accumulator buffers in the 512 TMEM columns: the normal variant's 256-column tiles
 // take two; the swap-AB variant's tiles are at most 64 columns (chunk_rows <= 64), so it
-// keeps eight, letting the epilogue (stores, split-K hand-off) lag up to seven tiles.
+// keeps eight, letting the epilogue (stores, split-K hand-off) lag up to seven tiles; its
+// wide form (chunk_rows <= 128, for batches whose heavy experts would otherwise stream the
+// same weight tiles once per 64-row chunk) keeps four of 128 columns.
 constexpr int kMaxAccStages = 8;
-template <bool kSwap> struct AccLayout {
-  static constexpr int kStages = kSwap ? 8 : 2;
-  static constexpr int kCols = kSwap ? 64 : 256;
+template <bool kSwap, bool kWide = false> struct AccLayout {
+  static constexpr int kStages = kSwap ? (kWide ? 4 : 8) : 2;
+  static constexpr int kCols = kSwap ? (kWide ? 128 : 64) : 256;
 };
 constexpr int kTmemCols = 512;
 constexpr int kSmemBudget = 220 * 1024;
@@ -100,8 +102,9 @@ __device__ __forceinline__ Unit decode_unit(long u, const Chunk* chunks, int per
   return t;
 }
 
-template <bool kFp8, bool kSwap, int kGemm>
+template <bool kFp8, bool kSwap, int kGemm, bool kWide>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs a) {
+  using Acc = AccLayout<kSwap, kWide>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ SmemCtl ctl;
 
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
-    for (int i = 0; i < AccLayout<kSwap>::kStages; ++i) {
+    for (int i = 0; i < Acc::kStages; ++i) {
       mbar_init(&ctl.tmem_full[i], 1);
       mbar_init(&ctl.tmem_empty[i], 4);
     }
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * AccLayout<kSwap>::kCols);
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * Acc::kCols);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&ctl.full[stage], phase, abort_flag, a.status, budget)) {
             ok = false;
@@ -328,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
         if (!ok) break;
         tc_commit(&ctl.tmem_full[acc]);
-        if (++acc == AccLayout<kSwap>::kStages) {
+        if (++acc == Acc::kStages) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -355,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const uint32_t tb =
-          tmem_base + static_cast<uint32_t>(acc * AccLayout<kSwap>::kCols) + (static_cast<uint32_t>(q * 32) << 16);
+          tmem_base + static_cast<uint32_t>(acc * Acc::kCols) + (static_cast<uint32_t>(q * 32) << 16);
       if constexpr (kSwap && kGemm == 1) {
         // lane r of quarter q: gate (r%32 < 16) or up (r%32 >= 16) of feature
         // tile*64 + 16q + r%16; column c = token row0 + c
@@ -471,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.tmem_empty[acc]);
-      if (++acc == AccLayout<kSwap>::kStages) {
+      if (++acc == Acc::kStages) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -497,13 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   }
 }
 
-template <bool kFp8, bool kSwap, int kGemm>
+template <bool kFp8, bool kSwap, int kGemm, bool kWide = false>
 cudaError_t launch_one(const GemmArgs& a, int num_sms, cudaStream_t s) {
+  if (kSwap && !kWide && a.chunk_rows > 64) return launch_one<kFp8, kSwap, kGemm, true>(a, num_sms, s);
+  if (a.chunk_rows > AccLayout<kSwap, kWide>::kCols) return cudaErrorInvalidValue;
   const int stage_bytes = kTileA + (kSwap ? a.chunk_rows * 128 : 2 * kTileA);
   const size_t smem = 1024 + static_cast<size_t>(a.nstages) * stage_bytes;
-  cudaError_t err = set_max_dynamic_smem<gemm_kernel<kFp8, kSwap, kGemm>>(kSmemBudget + 1024);
+  cudaError_t err = set_max_dynamic_smem<gemm_kernel<kFp8, kSwap, kGemm, kWide>>(kSmemBudget + 1024);
   if (err != cudaSuccess) return err;
-  return launch_k(gemm_kernel<kFp8, kSwap, kGemm>, dim3(num_sms), dim3(kThreads), smem, s, a);
+  return launch_k(gemm_kernel<kFp8, kSwap, kGemm, kWide>, dim3(num_sms), dim3(kThreads), smem, s, a);
 }
 
 }  // namespace

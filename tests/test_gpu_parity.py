@@ -281,8 +281,8 @@ def test_out_of_range_expert_ids_are_reported(small_cases):
 FULL = [("mixtral_fp8_decode", T) for T in (1, 8, 32, 64)] + \
        [("dsv3_fp8_decode", T) for T in (16, 64, 256)] + \
        [("swapab_stress_fp8", 8), ("swapab_adversarial_fp8", 8), ("prefill_fp8", 4096)] + \
-       [("mixtral_bf16_decode", T) for T in (8, 64)] + [("prefill_bf16", 4096)] + \
-       [("dsv3_grouped_fp8_decode", 64)]
+       [("mixtral_bf16_decode", T) for T in (1, 8, 64)] + [("prefill_bf16", 4096)] + \
+       [("dsv3_grouped_fp8_decode", T) for T in (16, 64, 256)]
 
 
 @pytest.fixture(scope="module")
