@@ -352,13 +352,17 @@ FMOE_API fmoe_status fused_inv_rope_fp8_quant_per_head(const fmoe_rope_dims* dim
  * workspace: the workspace is a file-scope device array of FUSED_MOE_STATIC_WS_BYTES
  * that the library owns, and every GPU that loads the library holds it until the
  * process exits.  It allocates nothing.
- *   - Dims whose fused_moe_workspace_size exceeds FUSED_MOE_STATIC_WS_BYTES are
- *     rejected with FMOE_ERR_WORKSPACE (use fused_moe with your own workspace).
- *   - The first call on each device, with that device current, looks up the array's
- *     device address; make that first call before any stream capture.
+ *   - Every argument check of fused_moe runs first, with its status codes, then dims
+ *     whose fused_moe_workspace_size exceeds FUSED_MOE_STATIC_WS_BYTES are rejected with
+ *     FMOE_ERR_WORKSPACE (use fused_moe with your own workspace); no CUDA call happens
+ *     before these checks.
+ *   - Every call looks up the array's device address in the current context (a host-side
+ *     lookup that enqueues nothing); the first call in a context loads the library's
+ *     module there, so make it before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents; each call
- *     clears the workspace header (device status word) first.  Calls that overlap on
- *     the GPU race on the array: the caller must serialise them.
+ *     first clears what fused_moe_workspace_init clears (the status word and the
+ *     router's tile counters).  Calls that overlap on the GPU race on the array: the
+ *     caller must serialise them.
  *   - device_status (device pointer to one int32, 4-byte aligned, may be NULL)
  *     receives this call's device status word (FMOE_OK, FMOE_ERR_TIMEOUT or
  *     FMOE_ERR_DEVICE_BOUNDS) when the stream reaches the end of the call. */
