@@ -160,6 +160,8 @@ SMALL = [
     ("bf16_router_tiled_e130", (1000, 512, 128, 130, 3, "bf16"), {}),
     ("fp8_router_tiled_grouped", (1600, 512, 128, 64, 6, "fp8"),
      {"router_std": 1.0, "grouped": (8, 3, 2.5), "n_shared": 1}),
+    # more than 32 slots per token: the swap-AB output is combined by its own launch
+    ("fp8_many_slots", (6, 256, 128, 40, 34, "fp8"), {}),
 ]
 
 
@@ -244,6 +246,55 @@ def test_static_scales(small_cases, variant):
     assert np.array_equal(gpu["a_perm"], ref["a_perm"])
     assert gpu["scalars"]["s1"] == np.float32(0.02) and gpu["scalars"]["s2"] == np.float32(0.003)
     check_layer(gpu, ref, "fp8")
+
+
+@pytest.mark.parametrize("name,launches", [
+    # T=1: router (+ permutation, plan, gather), the split-K first contraction, its finish,
+    # the quantisation of h, the second contraction, the finish + combine of its partials
+    ("fp8_single_token", ["router_permute_gather", "gemm1_swapab", "finalize1", "quant_h",
+                          "gemm2_swapab", "combine_partials"]),
+    ("fp8_ragged", ["router_permute_gather", "gemm1_swapab", "finalize1", "quant_h",
+                    "gemm2_swapab", "combine_partials"]),
+    # 34 slots per token
+    ("fp8_many_slots", ["router_permute_gather", "gemm1_swapab", "finalize1", "quant_h",
+                        "gemm2_swapab", "combine_partials"]),
+    ("bf16_shared_two", ["router_permute_gather", "gemm1_swapab", "finalize1", "gemm2_swapab",
+                         "combine_partials"]),
+    ("fp8_grouped_shared", None),
+])
+def test_swap_repeat_and_reinit(small_cases, name, launches):
+    """Repeated swap-AB calls on one workspace, with its header re-initialised in between
+    or not, give identical bits, within tolerance of the oracle and equal to the
+    step-by-step path (separate finish and combine); the launch list of a profiled call is
+    the documented one and as long as fused_moe_launches_per_call says."""
+    inp, g, ref = small_cases(name)
+    s = inp.shape
+    dims = capi.make_dims(s.T, s.H, s.I, s.E, s.top_k, s.wdtype == "fp8", "swap_ab",
+                          routing=g.get("routing"))
+    ws = capi.alloc_workspace(dims)
+    sc = capi.make_scales(g["w13_scale"], g["w2_scale"])
+    outs = []
+    for i in range(4):
+        if i == 2:
+            capi.fused_moe_workspace_init(ws)
+        out = torch.full((s.T, s.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        capi.fused_moe(dims, g["x"], g["router_w"], g["w13"], g["w2"], sc, out, ws)
+        torch.cuda.synchronize()
+        assert capi.fused_moe_get_device_status(ws) == capi.FMOE_OK
+        outs.append(bits16(out))
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    assert max_rel_err(bf16_bits_to_float(outs[0]), ref["out64"]) <= TOL[s.wdtype]
+    steps = run_steps(inp, g, "swap_ab")
+    assert np.array_equal(outs[0], steps["out"])
+    if launches is not None:
+        out = torch.empty(s.T, s.H, dtype=torch.bfloat16, device="cuda")
+        got = [n for n, _ in capi.fused_moe_profile(dims, g["x"], g["router_w"], g["w13"],
+                                                    g["w2"], sc, out, ws)]
+        assert got == launches
+        assert len(got) == capi.fused_moe_launches_per_call(dims)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits16(out), outs[0])
 
 
 def test_host_io_matches_device_call(small_cases):
