@@ -17,8 +17,10 @@
 // One CTA (8 warps) handles TB tokens.  Their x rows are staged in shared memory with
 // 16-byte loads; each warp takes groups of EG experts and streams the router rows from
 // L2, so each x chunk read from shared memory feeds 8*EG FMAs.  Top-k is then one warp
-// per token: k rounds of a shuffle argmax over (logit desc, expert index asc); shared
-// experts, when present, fill the token's last slots with weight 1.
+// per token: k rounds of a warp argmax over (logit desc, expert index asc), each two
+// redux.sync reductions; lane r keeps the weight of choice r, so the k weights are
+// normalised by k lanes at once.  Shared experts, when present, fill the token's last slots
+// with weight 1.
 #include <float.h>
 
 #include "permute_body.cuh"
@@ -43,6 +45,21 @@ __device__ __forceinline__ bool better(float av, int ae, float bv, int be) {
   return av > bv || (av == bv && ae < be);
 }
 
+// Warp-wide best candidate: the largest v, ties to the smallest e -- the pair a pairwise
+// reduction with better() keeps -- in two warp reductions (redux.sync) instead of five
+// shuffle rounds.  Scores map to unsigned keys that order like the floats (-0 counted as
+// +0, as float comparison does; NaN never occurs here).  Every lane gets the result.
+__device__ __forceinline__ void warp_best(float& v, int& e) {
+  uint32_t b = __float_as_uint(v);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t key = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+  const uint32_t emin =
+      __reduce_min_sync(0xffffffffu, key == kmax ? static_cast<uint32_t>(e) : 0xffffffffu);
+  v = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax);
+  e = static_cast<int>(emin);
+}
+
 // Affinity of the grouped router: sigmoid evaluated in fp64, rounded once to fp32.
 __device__ __forceinline__ float sigmoid_f64(float l) {
   return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(l))));
@@ -64,10 +81,11 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
   const int E = a.E;
   if (split) {
     // The last of the gridDim.y CTAs of this token tile to finish picks the top-k
-    // (counter reset for the next call by that CTA).
-    __threadfence();  // every writer orders its logits before the hand-off
+    // (counter reset for the next call by that CTA).  The barrier orders every thread's
+    // logits before thread 0's gpu-scope fence, whose release covers them (cumulativity).
     __syncthreads();
     if (threadIdx.x == 0) {
+      __threadfence();
       const int prev = atomicAdd(&a.tile_counters[tile], 1);
       is_last = prev == static_cast<int>(gridDim.y) - 1;
       if (is_last) {
@@ -91,16 +109,18 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
     const int tok = t0 + t;
     if (tok >= a.T) break;
     constexpr int kPer = kMaxExperts / 32;
-    float v[kPer];
+    float v[kPer], aff[kPer];  // selection scores; grouped: the unbiased affinities
     bool taken[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int e = lane + 32 * j;
       float l = -INFINITY;
+      aff[j] = 0.f;
       if (e < E) {
         l = logits[t * E + e];
         if (grouped) {
-          l = sigmoid_f64(l) + (a.bias != nullptr ? a.bias[e] : 0.f);
+          aff[j] = sigmoid_f64(l);
+          l = aff[j] + (a.bias != nullptr ? a.bias[e] : 0.f);
           sbs[t * E + e] = l;
         }
       }
@@ -132,12 +152,7 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
       for (int r = 0; r < a.topk_group; ++r) {
         float bv = gtaken ? -INFINITY : gs;
         int be = gtaken ? 0x7fffffff : lane;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-          if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-        }
+        warp_best(bv, be);
         keep |= 1u << be;
         if (lane == be) gtaken = true;
       }
@@ -151,6 +166,8 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
     const int K = a.k + a.n_shared;  // slots per token: k routed, then the shared experts
     float* wout = a.topk_w + static_cast<size_t>(tok) * K;
     int32_t* iout = a.topk_ids + static_cast<size_t>(tok) * K;
+    float my_ex = 0.f;  // lane r < 32 keeps the weight and expert of choice r
+    int my_e = 0;
     for (int r = 0; r < a.k; ++r) {
       float bv = -INFINITY;
       int be = 0x7fffffff;
@@ -159,42 +176,53 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
         const int e = lane + 32 * j;
         if (!taken[j] && better(v[j], e, bv, be)) { bv = v[j]; be = e; }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-      }
+      warp_best(bv, be);
+      float mine = 0.f;
 #pragma unroll
       for (int j = 0; j < kPer; ++j)
-        if (lane + 32 * j == be) taken[j] = true;
+        if (lane + 32 * j == be) {
+          taken[j] = true;
+          mine = aff[j];
+        }
       float ex;
       if (grouped) {
-        ex = sigmoid_f64(logits[t * E + be]);  // the unbiased affinity of the j-th choice
+        ex = __shfl_sync(0xffffffffu, mine, be & 31);  // the unbiased affinity of the choice
       } else {
         if (r == 0) top0 = bv;
         ex = expf(bv - top0);  // exp(l_j - l_max) of the j-th choice
       }
       wsum += ex;  // summed in choice order
-      if (lane == 0) { iout[r] = be; wout[r] = ex; }
-    }
-    if (lane == 0) {
-      const float scale = grouped ? a.routed_scaling : 1.f;
-      for (int r = 0; r < a.k; ++r) wout[r] = grouped ? wout[r] / wsum * scale : wout[r] / wsum;
-      // shared experts: every token, weight exactly 1, after the routed slots
-      for (int r = 0; r < a.n_shared; ++r) {
-        iout[a.k + r] = a.E + r;
-        wout[a.k + r] = 1.f;
+      if (r < 32) {
+        if (lane == r) {
+          my_ex = ex;
+          my_e = be;
+        }
+      } else if (lane == 0) {
+        iout[r] = be;
+        wout[r] = ex;
       }
+    }
+    // the k weights normalised lane-parallel (choices past 32 went through memory)
+    const float scale = grouped ? a.routed_scaling : 1.f;
+    if (lane < a.k) {
+      iout[lane] = my_e;
+      wout[lane] = grouped ? my_ex / wsum * scale : my_ex / wsum;
+    }
+    __syncwarp();
+    for (int r = 32 + lane; r < a.k; r += 32) wout[r] = grouped ? wout[r] / wsum * scale : wout[r] / wsum;
+    // shared experts: every token, weight exactly 1, after the routed slots
+    for (int r = lane; r < a.n_shared; r += 32) {
+      iout[a.k + r] = a.E + r;
+      wout[a.k + r] = 1.f;
     }
   }
 
   if (a.fuse_permute) {
     // The CTA that finishes the last token tile groups the rows by expert (and plans
     // the GEMMs, and for small batches gathers the activations) for the whole batch.
-    __threadfence();  // this CTA's top-k results (and max |x|) before the hand-off
-    __syncthreads();
+    __syncthreads();  // this CTA's top-k results (and max |x|), published by thread 0's fence
     if (threadIdx.x == 0) {
+      __threadfence();
       const int prev = atomicAdd(a.route_done, 1);
       is_final = prev == static_cast<int>(gridDim.x) - 1;  // one top-k CTA per tile
       if (is_final) {
@@ -360,6 +388,8 @@ constexpr int kRtSlice = 256;                 // columns per slice
 constexpr int kRtRowBytes = kRtSlice * 2;     // bf16
 constexpr uint64_t kRtBudgetNs = 2000000000ull;
 constexpr int kRtLogitsOff = 32 * 1024;       // logits after the permutation scratch
+constexpr int kRtTokensPerWarp32 = 4;         // tokens per warp of the 16 x 32 tile (8, with
+                                              // half the warps, measured 8-12% slower)
 
 template <int N>
 __device__ __forceinline__ void halve(float (&v)[32], int lane) {
@@ -383,23 +413,22 @@ template <int TBC, int ECC>
 constexpr size_t rt_stage_bytes() { return static_cast<size_t>(TBC + ECC) * kRtRowBytes; }
 
 // Warps of the tiled router: (ECC / 8) expert groups x as many token groups as give each
-// warp 4 tokens, i.e. 32 accumulators per lane.
-template <int TBC, int ECC>
-constexpr int rt_warps() { return (ECC / 8) * (TBC / 4); }
+// warp TBW tokens, i.e. 8 * TBW accumulators per lane.
+template <int TBC, int ECC, int TBW>
+constexpr int rt_warps() { return (ECC / 8) * (TBC / TBW); }
 
-template <int TBC, int ECC>
-__global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
+template <int TBC, int ECC, int TBW>
+__global__ void __launch_bounds__(rt_warps<TBC, ECC, TBW>() * 32, 1)
     router_tiled_kernel(const __grid_constant__ RouterArgs a, const __grid_constant__ RouterMaps m) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[kRtStages];
   __shared__ __align__(8) uint64_t empty[kRtStages];
   __shared__ int abort_flag;
   __shared__ uint32_t amax_bits;
-  constexpr int NW = rt_warps<TBC, ECC>();
+  constexpr int NW = rt_warps<TBC, ECC, TBW>();
   constexpr int NTHR = NW * 32;
   constexpr int NG = ECC / 8;        // groups of 8 experts in the tile
-  constexpr int TBW = 4;             // tokens per warp
-  static_assert(NG * (TBC / TBW) == NW, "warp tiling");
+  static_assert(TBW % 4 == 0 && NG * (TBC / TBW) == NW, "warp tiling");
   constexpr uint32_t kStageBytes = static_cast<uint32_t>(rt_stage_bytes<TBC, ECC>());
 
   const uint32_t raw = smem_u32(smem_raw);
@@ -524,16 +553,17 @@ __global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
   // ---- butterfly over lanes for the warp's 32 logits, into smem or the split buffer
   float* logits = reinterpret_cast<float*>(smem + kRtLogitsOff);  // [TBC][E] (+ scores)
   const int e_end = min(a.E, e0 + ECC);
-  {
+#pragma unroll
+  for (int pass = 0; pass < TBW / 4; ++pass) {  // 32 logits (4 tokens x 8 experts) per pass
     float v[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = acc[j / 8][j % 8];
+    for (int j = 0; j < 32; ++j) v[j] = acc[4 * pass + j / 8][j % 8];
     halve<32>(v, lane);
     halve<16>(v, lane);
     halve<8>(v, lane);
     halve<4>(v, lane);
     halve<2>(v, lane);
-    const int tl = tg * TBW + lane / 8;  // token within the tile
+    const int tl = tg * TBW + 4 * pass + lane / 8;  // token within the tile
     const int e = e0 + eg * 8 + (lane & 7);
     if (e < e_end) {
       if (split) {
@@ -551,10 +581,10 @@ __global__ void __launch_bounds__(rt_warps<TBC, ECC>() * 32, 1)
   router_tail<TBC, NTHR>(a, smem, logits, tile, split);
 }
 
-template <int TBC, int ECC>
+template <int TBC, int ECC, int TBW>
 cudaError_t launch_tiled(const RouterArgs& a0, const RouterMaps& m, cudaStream_t s) {
   RouterArgs a = a0;
-  constexpr int NTHR = rt_warps<TBC, ECC>() * 32;
+  constexpr int NTHR = rt_warps<TBC, ECC, TBW>() * 32;
   constexpr size_t ring = kRtStages * rt_stage_bytes<TBC, ECC>();
   const size_t need = kRtLogitsOff + static_cast<size_t>(TBC) * a.E * 4 * 2;
   if (a.fuse_permute) {  // permute_body's scratch sits below the logits
@@ -562,12 +592,12 @@ cudaError_t launch_tiled(const RouterArgs& a0, const RouterMaps& m, cudaStream_t
     if (perm > kRtLogitsOff) return cudaErrorInvalidValue;  // cannot happen: E_all <= 264
   }
   const size_t smem = 1024 + (ring > need ? ring : need);
-  cudaError_t err = set_max_dynamic_smem<router_tiled_kernel<TBC, ECC>>(static_cast<int>(smem));
+  cudaError_t err = set_max_dynamic_smem<router_tiled_kernel<TBC, ECC, TBW>>(static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int tiles = (a.T + TBC - 1) / TBC;
   const int groups = (a.E + ECC - 1) / ECC;
   a.experts_per_cta = groups == 1 ? a.E : ECC;
-  return launch_k(router_tiled_kernel<TBC, ECC>, dim3(tiles, groups), dim3(NTHR), smem, s, a, m);
+  return launch_k(router_tiled_kernel<TBC, ECC, TBW>, dim3(tiles, groups), dim3(NTHR), smem, s, a, m);
 }
 
 template <int TB, int EG>
@@ -624,8 +654,8 @@ bool router_use_tiled(int T, int E, int num_sms) {
 }
 
 cudaError_t launch_router_tiled(const RouterArgs& a, const RouterMaps& m, cudaStream_t s) {
-  if (a.E <= 8) return launch_tiled<32, 8>(a, m, s);
-  return launch_tiled<16, 32>(a, m, s);
+  if (a.E <= 8) return launch_tiled<32, 8, 4>(a, m, s);
+  return launch_tiled<16, 32, kRtTokensPerWarp32>(a, m, s);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
