@@ -319,7 +319,7 @@ PermuteArgs permute_args(const fmoe_dims& d, const Layout& L, const int32_t* ids
                          const fmoe_scales* sc, int32_t* counts, int32_t* offsets, int32_t* rows,
                          int32_t* inv, char* W, bool with_plan);
 GatherArgs gather_args(const fmoe_dims& d, const Layout& L, const void* x, const int32_t* rows,
-                       void* a_perm, char* W);
+                       const int32_t* inv, void* a_perm, char* W);
 
 fmoe_status route_impl(const fmoe_dims& d, const Layout& L, const void* x, const void* rw,
                        int32_t* ids, float* tw, char* W, cudaStream_t s,
@@ -397,11 +397,12 @@ PermuteArgs permute_args(const fmoe_dims& d, const Layout& L, const int32_t* ids
 }
 
 GatherArgs gather_args(const fmoe_dims& d, const Layout& L, const void* x, const int32_t* rows,
-                       void* a_perm, char* W) {
+                       const int32_t* inv, void* a_perm, char* W) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(W + L.hdr);
   GatherArgs g{};
   g.x = static_cast<const uint16_t*>(x);
   g.sorted_rows = rows;
+  g.inv_perm = inv;
   g.a_perm = a_perm;
   g.hdr = hdr;
   g.status = &hdr->status;
@@ -418,7 +419,7 @@ fmoe_status permute_impl(const fmoe_dims& d, const Layout& L, const int32_t* ids
   const NvtxRange range("fused_moe.permute");
   const PermuteArgs p = permute_args(d, L, ids, sc, counts, offsets, rows, inv, W, with_plan);
   FMOE_LAUNCH(with_plan ? "permute_plan" : "permute", launch_permute(p, s), s);
-  const GatherArgs g = gather_args(d, L, x, rows, a_perm, W);
+  const GatherArgs g = gather_args(d, L, x, rows, inv, a_perm, W);
   FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);
   return FMOE_OK;
 }
@@ -653,7 +654,7 @@ fmoe_status first_half(const fmoe_dims& d, const Layout& L, const OneCall& b, co
   bool plan_two_back = true;  // the plan-writing launch is followed by the gather launch
   if (fuse_route_permute(L)) {
     const PermuteArgs p = permute_args(d, L, b.ids, sc, b.counts, b.offsets, b.rows, b.inv, W, true);
-    const GatherArgs g = gather_args(d, L, x, b.rows, W + L.a_perm, W);
+    const GatherArgs g = gather_args(d, L, x, b.rows, b.inv, W + L.a_perm, W);
     const bool fg = fuse_route_gather(d, L);
     FMOE_TRY(route_impl(d, L, x, rw, b.ids, b.tw, W, s, &p, fg ? &g : nullptr));
     if (!fg) FMOE_LAUNCH("gather_quant", launch_gather(g, s), s);

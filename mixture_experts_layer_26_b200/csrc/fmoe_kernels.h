@@ -82,6 +82,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 struct GatherArgs {
   const uint16_t* x;          // [T, H] bf16
   const int32_t* sorted_rows; // [R]
+  const int32_t* inv_perm;    // [R]: permuted row of each (token, slot)
   void* a_perm;               // [R, H] e4m3 bytes or bf16
   const WsHeader* hdr;        // inv1
   int32_t* status;

@@ -16,7 +16,8 @@
 //   gives s and 1/s).
 // gather_kernel: A[p] = x[sorted_rows[p] / k], read with 16-byte loads and, for the
 //   FP8 format, multiplied by the inverse scale in fp32 and rounded to e4m3
-//   (round to nearest even, saturating at +-448).
+//   (round to nearest even, saturating at +-448); token-major (each x row read once and
+//   stored to its k rows p = inv_perm[t*k + j]).
 // plan_kernel (one warp): splits every expert's rows into chunks of at most
 //   chunk_rows rows and picks split-K factors for the swap-AB contractions.
 #include "permute_body.cuh"
@@ -59,8 +60,10 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
-  const int rows_per_block = kGatherThreads / 32;
-  int grid = (a.R + rows_per_block - 1) / rows_per_block;
+  const int warps_per_block = kGatherThreads / 32;
+  const int steps = a.fp8 ? a.H / 16 : a.H / 8;
+  const long items = static_cast<long>(a.R / a.k) * ((steps + 32 * kGatherU - 1) / (32 * kGatherU));
+  int grid = static_cast<int>((items + warps_per_block - 1) / warps_per_block);
   grid = grid < 1 ? 1 : grid;
   return launch_k(gather_kernel, dim3(grid), dim3(kGatherThreads), 0, s, a);
 }

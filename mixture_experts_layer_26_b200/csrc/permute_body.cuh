@@ -18,8 +18,10 @@ __device__ int choose_split(int units, int kblocks, int smax, int sms) {
   int best = 1;
   float best_eff = -1.f;
   for (int s = 1; s <= cap; ++s) {
-    const long u = static_cast<long>(units) * s;
-    const long waves = (u + sms - 1) / sms;
+    // 32-bit arithmetic (units * 16 stays far below 2^31): a 64-bit division is a long
+    // serial call on the one thread that plans
+    const int u = units * s;
+    const int waves = (u + sms - 1) / sms;
     const float eff = static_cast<float>(u) / static_cast<float>(waves * sms);
     if (eff >= 0.9f) return s;
     if (eff > best_eff + 1e-6f) { best_eff = eff; best = s; }
@@ -260,43 +262,72 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
 // Rows p = gwarp, gwarp + nwarps, ... of the permuted activations, one warp per row:
 // A[p] = x[sorted_rows[p] / k] with 16-byte loads, FP8: times 448/amax in fp32, rounded
 // to e4m3 (nearest even, saturating).
+// Token-major gather: a warp takes one (token, segment of up to 32*kGatherU 16-byte steps)
+// item, reads that part of the token's x row once, quantises it once (FP8), and stores it to
+// each of the token's k permuted rows p = inv_perm[t*k + j] (lane j holds slot j's row when
+// k <= 32).  Every permuted row gets exactly the bytes a row-major gather would write; x is
+// read once instead of k times.
+constexpr int kGatherU = 4;  // 16-byte steps per lane and item
+
+__device__ __forceinline__ int gather_items(const GatherArgs& a) {
+  const int steps = a.fp8 ? a.H / 16 : a.H / 8;  // FP8: 16 elements; bf16: 8 per step
+  return (a.R / a.k) * ((steps + 32 * kGatherU - 1) / (32 * kGatherU));
+}
+
 __device__ void gather_rows(const GatherArgs& a, int gwarp, int nwarps) {
   const int lane = threadIdx.x & 31;
   const float inv = a.fp8 ? a.hdr->inv1 : 1.f;
-  const int nvec = a.H / 16;  // 16 elements per step
-  for (int p = gwarp; p < a.R; p += nwarps) {
-    const int r = a.sorted_rows[p];
-    if (r < 0 || r >= a.R) {
-      if (lane == 0) record_status(a.status, ST_BOUNDS);
-      continue;
-    }
-    const int t = r / a.k;
+  const int k = a.k;
+  const int steps = a.fp8 ? a.H / 16 : a.H / 8;
+  const int nseg = (steps + 32 * kGatherU - 1) / (32 * kGatherU);
+  const int items = gather_items(a);
+  for (int it = gwarp; it < items; it += nwarps) {
+    const int t = it / nseg, s0 = (it % nseg) * 32 * kGatherU;
+    auto row_of = [&](int j) {  // permuted row of slot j, -1 if out of range (reported)
+      int p = a.inv_perm[static_cast<size_t>(t) * k + j];
+      if (p < 0 || p >= a.R) {
+        record_status(a.status, ST_BOUNDS);
+        p = -1;
+      }
+      return p;
+    };
+    const int pl = lane < k ? row_of(lane) : -1;
     const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H);
+    uint4 v[kGatherU];
     if (a.fp8) {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);
-      constexpr int kU = 4;  // 128 bytes of x per lane in flight
-      for (int v0 = lane; v0 < nvec; v0 += 32 * kU) {
-        uint4 x0[kU], x1[kU];
+      uint4 x0[kGatherU], x1[kGatherU];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nvec) {
-            x0[u] = __ldg(src + 2 * v);
-            x1[u] = __ldg(src + 2 * v + 1);
-          }
+      for (int u = 0; u < kGatherU; ++u) {
+        const int st = s0 + lane + 32 * u;
+        if (st < steps) {
+          x0[u] = __ldg(src + 2 * st);
+          x1[u] = __ldg(src + 2 * st + 1);
         }
+      }
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nvec) {
-            const uint2 q0 = quant8(x0[u], inv), q1 = quant8(x1[u], inv);
-            dst[v] = make_uint4(q0.x, q0.y, q1.x, q1.y);
-          }
+      for (int u = 0; u < kGatherU; ++u) {
+        if (s0 + lane + 32 * u < steps) {
+          const uint2 q0 = quant8(x0[u], inv), q1 = quant8(x1[u], inv);
+          v[u] = make_uint4(q0.x, q0.y, q1.x, q1.y);
         }
       }
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.a_perm) + static_cast<size_t>(p) * a.H);
-      for (int v = lane; v < 2 * nvec; v += 32) dst[v] = __ldg(src + v);
+#pragma unroll
+      for (int u = 0; u < kGatherU; ++u) {
+        const int st = s0 + lane + 32 * u;
+        if (st < steps) v[u] = __ldg(src + st);
+      }
+    }
+    const size_t row_bytes = static_cast<size_t>(a.H) * (a.fp8 ? 1 : 2);
+    for (int j = 0; j < k; ++j) {
+      const int p = j < 32 ? __shfl_sync(0xffffffffu, pl, j) : row_of(j);  // warp-uniform
+      if (p < 0) continue;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.a_perm) + static_cast<size_t>(p) * row_bytes);
+#pragma unroll
+      for (int u = 0; u < kGatherU; ++u) {
+        const int st = s0 + lane + 32 * u;
+        if (st < steps) dst[st] = v[u];
+      }
     }
   }
 }
