@@ -259,10 +259,14 @@ __global__ void __launch_bounds__(kEwThreads) combine_partials_kernel(CombinePar
         v0.x += u0.x; v0.y += u0.y; v0.z += u0.z; v0.w += u0.w;
         v1.x += u1.x; v1.y += u1.y; v1.z += u1.z; v1.w += u1.w;
       }
-      const float y[8] = {v0.x * sc * wr, v0.y * sc * wr, v0.z * sc * wr, v0.w * sc * wr,
-                          v1.x * sc * wr, v1.y * sc * wr, v1.z * sc * wr, v1.w * sc * wr};
+      // explicitly rounded products and sums: a multiply-add fused by the compiler here
+      // would not match finalize2 (which stores y) followed by combine
+      const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = (j == 0) ? y[i] : acc[i] + y[i];
+      for (int i = 0; i < 8; ++i) {
+        const float y = __fmul_rn(__fmul_rn(vv[i], sc), wr);
+        acc[i] = (j == 0) ? y : __fadd_rn(acc[i], y);
+      }
     }
     store_out(a.out, a.out_f32, static_cast<size_t>(t) * a.H + c, acc);
   }
