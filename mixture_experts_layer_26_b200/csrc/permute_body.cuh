@@ -113,9 +113,12 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float inv) {
 // in ascending order, so rows of one expert keep their flattened order (t*k+j).
 // Runs on a whole CTA of kWarps warps.  wc: kWarps*E ints, cnt: E, base: E+1 (shared).
 // Reads ids and amax partials through L2 (__ldcg): when fused into the router they were
-// written by other CTAs of the same grid.
+// written by other CTAs of the same grid.  n_parts > 0: the number of max |x| partials (the
+// router's grid, when fused into it) instead of the header's count; inv_s (shared, or null)
+// also receives the inverse activation scale, for a gather in the same CTA.
 template <int kWarps>
-__device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* base) {
+__device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* base,
+                             int n_parts = 0, float* inv_s = nullptr) {
   constexpr int kPermThreads = kWarps * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E, R = a.R;
@@ -142,10 +145,16 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
     }
   };
 
-  // pass 1: rows per (warp, expert)
+  // pass 1: rows per (warp, expert); a segment of one batch keeps its ids for pass 2
+  const bool one_batch = hi - lo <= 32 * kBatch;
+  int ev_kept[kBatch];
   for (int i0 = lo; i0 < hi; i0 += 32 * kBatch) {
     int ev[kBatch];
     load_batch(i0, ev);
+    if (one_batch) {
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) ev_kept[j] = ev[j];
+    }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       if (i0 + 32 * j >= hi) break;  // warp-uniform
@@ -197,7 +206,7 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
   if (warp == 1) {
     // activation scale from the router's per-tile maxima (one warp, strided)
     float amax = 0.f;
-    const int n = __ldcg(&a.hdr->router_ctas);
+    const int n = n_parts > 0 ? n_parts : __ldcg(&a.hdr->router_ctas);
     for (int i0 = lane; i0 < n; i0 += 32 * 8) {  // eight loads in flight per lane
       float v[8];
 #pragma unroll
@@ -221,6 +230,7 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
       a.hdr->amax_x = amax;
       a.hdr->s1 = s1;
       a.hdr->inv1 = inv1;
+      if (inv_s != nullptr) *inv_s = inv1;
     }
   }
   __syncthreads();
@@ -239,7 +249,12 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
   // pass 2: place every row, in ascending order within each warp's segment
   for (int i0 = lo; i0 < hi; i0 += 32 * kBatch) {
     int ev[kBatch];
-    load_batch(i0, ev);
+    if (one_batch) {
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) ev[j] = ev_kept[j];
+    } else {
+      load_batch(i0, ev);
+    }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       if (i0 + 32 * j >= hi) break;  // warp-uniform
@@ -274,9 +289,9 @@ __device__ __forceinline__ int gather_items(const GatherArgs& a) {
   return (a.R / a.k) * ((steps + 32 * kGatherU - 1) / (32 * kGatherU));
 }
 
-__device__ void gather_rows(const GatherArgs& a, int gwarp, int nwarps) {
+__device__ void gather_rows(const GatherArgs& a, int gwarp, int nwarps, const float* inv_s = nullptr) {
   const int lane = threadIdx.x & 31;
-  const float inv = a.fp8 ? a.hdr->inv1 : 1.f;
+  const float inv = a.fp8 ? (inv_s != nullptr ? *inv_s : a.hdr->inv1) : 1.f;
   const int k = a.k;
   const int steps = a.fp8 ? a.H / 16 : a.H / 8;
   const int nseg = (steps + 32 * kGatherU - 1) / (32 * kGatherU);

@@ -235,10 +235,12 @@ __device__ void router_tail(const RouterArgs& a, uint8_t* smem, float* logits, i
     // reuse: wc[8*Ea], cnt[Ea], base[Ea+1] over all Ea experts (shared ones included)
     const int Ea = a.perm.E;
     int* ps = reinterpret_cast<int*>(smem);
-    permute_body<NTHR / 32>(a.perm, ps, ps + (NTHR / 32) * Ea, ps + (NTHR / 32 + 1) * Ea);
+    __shared__ float inv1_s;  // the activation scale, handed from the permutation to the gather
+    permute_body<NTHR / 32>(a.perm, ps, ps + (NTHR / 32) * Ea, ps + (NTHR / 32 + 1) * Ea,
+                            static_cast<int>(gridDim.x), &inv1_s);
     if (a.fuse_gather) {
       __syncthreads();
-      gather_rows(a.gather, warp, NTHR / 32);
+      gather_rows(a.gather, warp, NTHR / 32, &inv1_s);
     }
   }
 }
