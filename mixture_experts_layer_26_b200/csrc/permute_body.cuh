@@ -274,9 +274,8 @@ __device__ void permute_body(const PermuteArgs& a, int* wc_flat, int* cnt, int* 
   }
 }
 
-// Rows p = gwarp, gwarp + nwarps, ... of the permuted activations, one warp per row:
-// A[p] = x[sorted_rows[p] / k] with 16-byte loads, FP8: times 448/amax in fp32, rounded
-// to e4m3 (nearest even, saturating).
+// The permuted activations A[p] = x[sorted_rows[p] / k], read with 16-byte loads; FP8:
+// times 448/amax in fp32, rounded to e4m3 (nearest even, saturating).
 // Token-major gather: a warp takes one (token, segment of up to 32*kGatherU 16-byte steps)
 // item, reads that part of the token's x row once, quantises it once (FP8), and stores it to
 // each of the token's k permuted rows p = inv_perm[t*k + j] (lane j holds slot j's row when
