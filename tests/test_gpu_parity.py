@@ -428,6 +428,56 @@ def test_router_full_shapes(workload, T):
             assert np.array_equal(got.cpu().numpy(), ref)
 
 
+TIE_CASES = [
+    # (T, H, E, k, grouped): the per-warp router with one, two and four experts per warp
+    # (E = 256: experts split over CTAs, handed to each token's last CTA), the tiled router
+    # with 32-token x 8-expert tiles and with expert groups handed to the tile's last CTA,
+    # and grouped sigmoid routing
+    (4, 512, 8, 2, None),
+    (37, 512, 64, 6, None),
+    (20, 1024, 256, 8, None),
+    (3000, 512, 8, 2, None),
+    (300, 512, 256, 8, None),
+    (64, 512, 64, 8, (8, 4, 2.5)),
+]
+
+
+@pytest.mark.parametrize("T,H,E,k,grouped", TIE_CASES)
+def test_router_ties_go_to_the_lower_expert(T, H, E, k, grouped):
+    """Exact ties in the selection: the upper half of the router rows repeats the lower half
+    (equal logits), two rows are zero (logit 0) and token 0 is zero (every logit 0, of either
+    sign): the chosen experts, in choice order, are the oracle's, which breaks every tie
+    towards the lower expert index, and the weights match."""
+    gen = torch.Generator().manual_seed(5)
+    x = torch.randn(T, H, generator=gen).to(torch.bfloat16)
+    x[0] = 0
+    wr = (torch.randn(E, H, generator=gen) / H ** 0.5).to(torch.bfloat16)
+    half = E // 2
+    wr[half:2 * half] = wr[:half]
+    wr[1] = 0
+    wr[half + 3] = 0
+    xb, wb = minp.bf16_bits(x), minp.bf16_bits(wr)
+    routing = None
+    if grouped is None:
+        ids_ref, w_ref, _ = O.router(xb, wb, k)
+    else:
+        ids_ref, w_ref, _, _ = O.router_grouped(xb, wb, k, n_group=grouped[0],
+                                                topk_group=grouped[1], routed_scaling=grouped[2])
+        routing = capi.make_routing(*grouped)
+    dims = capi.make_dims(T, H, 256, E, k, True, routing=routing)
+    ws = capi.alloc_workspace(dims)
+    ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    capi.fused_moe_route(dims, x.cuda(), wr.cuda(), ids, tw, ws)
+    torch.cuda.synchronize()
+    assert capi.fused_moe_get_device_status(ws) == capi.FMOE_OK
+    assert np.array_equal(ids.cpu().numpy().reshape(T, k), ids_ref)
+    assert np.allclose(tw.cpu().numpy().reshape(T, k), w_ref, rtol=1e-6, atol=1e-9)
+    # the ties are real: some token chose both copies of a duplicated router row
+    got = ids.cpu().numpy().reshape(T, k)
+    assert any(len(set(r) & {e + half for e in r if e < half}) > 0 for r in got)
+
+
 @pytest.mark.parametrize("name,variant", [("fp8_ragged", "swap_ab"), ("fp8_multichunk", "normal"),
                                           ("bf16_multichunk", "swap_ab"),
                                           ("fp8_pair_chunks", "normal_pair"),
