@@ -91,8 +91,10 @@ def profiled_traffic(kernel: str, workload_tag: str):
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
+    # the workload tag must be whole: "..._T1" must not match a summary of "..._T16"
+    tag = re.compile(re.escape(workload_tag) + r"(?=[._])")
     for name in sorted(os.listdir(pdir)):
-        if not (name.startswith(kernel) and workload_tag in name and name.endswith(".md")):
+        if not (name.startswith(kernel) and tag.search(name) and name.endswith(".md")):
             continue
         text = open(os.path.join(pdir, name)).read()
         t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)

@@ -54,3 +54,23 @@ def test_config_is_the_same_for_both_arms():
     for name in ("prefill_fp8", "dsv3_grouped_fp8_decode", "tiny_bf16"):
         cfg = bench.workload_config(minp.shape(name))
         assert "variant" not in cfg and cfg["workload"].startswith(name)
+
+
+def test_profiled_traffic_matches_whole_workload_tags(tmp_path, monkeypatch):
+    """The ncu summaries carry their DRAM traffic under a source hash; the lookup takes the
+    kernel's summary for exactly the workload and batch size asked for, and none whose hash
+    is not the current source's (synthetic summaries, so no real kernel source is involved)."""
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    for name, traffic, h in (("gemm1_swapab_mixtral_fp8_decode_T1.md", 111, "aa"),
+                             ("gemm1_swapab_mixtral_fp8_decode_T64.md", 6464, "aa"),
+                             ("gemm1_swapab_mixtral_fp8_decode_T16.md", 1616, "stale")):
+        (prof / name).write_text(f"traffic_bytes_per_launch: {traffic}\nsource_hash: {h}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "gemm_source_hash", lambda kernel="": "aa")
+    assert bench.profiled_traffic("gemm1_swapab", "mixtral_fp8_decode_T1") == 111
+    assert bench.profiled_traffic("gemm1_swapab", "mixtral_fp8_decode_T64") == 6464
+    assert bench.profiled_traffic("gemm1_swapab", "mixtral_fp8_decode_T6") is None
+    assert bench.profiled_traffic("gemm1_swapab", "mixtral_fp8_decode_T16") is None  # stale hash
+    assert bench.profiled_traffic("gemm2_swapab", "mixtral_fp8_decode_T1") is None
